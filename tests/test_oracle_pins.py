@@ -1,0 +1,52 @@
+"""The CPU oracle against hand cases, closed forms, a library special case,
+structure and invariants (no GPU)."""
+import numpy as np
+import pytest
+
+from oracle import brute
+from oracle import oracle as orc
+from tests import oracle_pins as pins
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return orc.load_library()
+
+
+@pytest.mark.parametrize("pin", pins.ALL_PINS, ids=lambda p: p.__name__)
+def test_pin(lib, pin):
+    pin(lib)
+
+
+@pytest.mark.parametrize("B,S,m,H,D,k,Tover", [
+    (1, 64, 4, 8, 64, 5, None),
+    (2, 50, 2, 4, 16, 30, None),
+    (1, 41, 3, 2, 8, 200, None),
+    (1, 24, 1, 16, 4, 3, 7),
+    (3, 20, 5, 1, 2, 2, 9),
+])
+def test_c_oracle_matches_numpy_restatement(lib, B, S, m, H, D, k, Tover):
+    """The C oracle and an independent numpy restatement agree exactly on
+    indices and to fp64 rounding on scores."""
+    rng = np.random.default_rng(S * 31 + k)
+    T = S // m if Tover is None else Tover
+    q = pins.random_bf16(rng, (B, S, H, D), scale=1 / np.sqrt(D))
+    w = rng.standard_normal((B, S, H)).astype(np.float32)
+    kc = pins.random_bf16(rng, (B, T, D))
+    idx, sc, _, _ = orc.topk_all_rows(q, w, kc, m, k, lib=lib)
+    bidx, bsc = brute.topk_all_rows(q, w, kc, m, k)
+    assert np.array_equal(idx, bidx)
+    fin = np.isfinite(bsc)
+    assert np.array_equal(np.isfinite(sc), fin)
+    assert np.allclose(sc[fin], bsc[fin], rtol=1e-12, atol=1e-12)
+
+
+def test_materialised_size_formula():
+    """Abstract: the [B,S,H_I,T] fp32 intermediate is 256 GB at S=65,536 with
+    H_I=64 and m=4 (T=S/m); 4*B*S*H_I*T bytes is exactly 2**38."""
+    S, H, m = 65536, 64, 4
+    assert 4 * 1 * S * H * (S // m) == 256 * 2**30
+
+
+def test_oracle_reports_threads(lib):
+    assert orc.max_threads() >= 1
