@@ -1,0 +1,392 @@
+"""Benchmark of the streaming top-k indexer step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload long] [--no-e2e] [--no-cpu-baseline]
+
+A step is one indexer call over one batch of synthetic inputs: the fused
+scoring + selection kernel and the per-row sort (what si_indexer_topk
+launches), with q, w, kc already resident in HBM.  Every rank runs its own
+problem of the named workload (seeds differ by rank), so per-GPU work is
+fixed as N grows ("scaling": "weak"); no data moves between ranks.
+
+Rank 0 prints one JSON line.  `value` is the indexer TFLOP/s of the whole
+job (2*H_I*d_I FLOPs per causally visible query-key pair, all ranks) over
+the device-timed region (max over ranks).  `--impl reference` times the CPU
+oracle (fp64, OpenMP) on bounded row samples of the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+METRIC = ("indexer TFLOP/s & query rows/s at S=262,144 (H_I=64,d_I=128,m=4,k=512); peak HBM")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def visible_pairs(B: int, S: int, T: int, m: int) -> int:
+    """Sum over query rows of min(T, floor((t+1)/m)) (closed form)."""
+    # rows with (t+1)//m < T contribute (t+1)//m; the rest contribute T
+    total = 0
+    full_from = m * T - 1  # first t with (t+1)//m >= T
+    n_part = min(S, max(full_from, 0))
+    # sum_{t=0}^{n_part-1} floor((t+1)/m) = sum_{x=1}^{n_part} floor(x/m)
+    x = n_part
+    q, r = divmod(x, m)
+    part = m * q * (q - 1) // 2 + q * (r + 1)
+    total = part + max(S - n_part, 0) * T
+    return B * total
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def csrc_hash() -> str:
+    d = os.path.join(ROOT, "streaming_top_indexer_b200", "csrc")
+    h = hashlib.sha256()
+    for name in sorted(os.listdir(d)):
+        if name.endswith((".cu", ".cuh")):
+            with open(os.path.join(d, name), "rb") as f:
+                h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(workload: str):
+    """DRAM bytes per launch of the select kernel from a committed ncu summary,
+    or None if absent or taken on different kernel sources."""
+    path = os.path.join(ROOT, "profiles", "select_kernel_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    if d.get("csrc_hash") != csrc_hash():
+        return None
+    return d.get("per_launch_bytes", {}).get(workload)
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during a region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{gpu_index}.csv")
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=self.fh, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sms, maxs, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sms.append(float(parts[1]))
+                    maxs.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for nm, v in zip(names, parts[5:9]):
+                    if v.lower().startswith("active"):
+                        reasons.add(nm)
+        if not sms:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        return {"sm_mhz": statistics.median(sms), "sm_max_mhz": max(maxs), "reasons": sorted(reasons),
+                "samples": len(sms)}
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if args.impl == "ours" else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=600))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def all_max(x: float, world: int, device) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def sample_rows_uniform(S: int, n: int, seed: int):
+    rng = np.random.default_rng(seed + 4242)
+    return np.sort(rng.choice(S, size=min(n, S), replace=False)).astype(np.int64)
+
+
+def oracle_sample(q, w, kc, wl, rows_t, b=0):
+    """Time the CPU oracle on the given rows of batch b; returns (seconds, flops)."""
+    from oracle import oracle as orc
+    from streaming_top_indexer_b200 import synth
+    tt = torch.from_numpy(rows_t).to(q.device)
+    q_rows = synth.bf16_bits(q[b, tt])
+    w_rows = w[b, tt].cpu().numpy()
+    kc_bits = synth.bf16_bits(kc[b:b + 1])
+    rb = np.zeros_like(rows_t)
+    t0 = time.perf_counter()
+    orc.topk_rows(q_rows, w_rows, rb, rows_t, kc_bits, wl.m, wl.k)
+    dt = time.perf_counter() - t0
+    vis = np.minimum(wl.T, (rows_t + 1) // wl.m)
+    flops = float(2 * wl.H * wl.D * vis.sum())
+    return dt, flops
+
+
+def cpu_baseline(q, w, kc, wl, budget_s: float, seed: int):
+    """Oracle on a bounded, seeded sample of the workload's rows (host cores)."""
+    from oracle import oracle as orc
+    cores = orc.max_threads()
+    # calibrate on a small sample, then size the main sample to the budget
+    probe = sample_rows_uniform(wl.S, max(cores, 8), seed)
+    dt, fl = oracle_sample(q, w, kc, wl, probe)
+    per_row = dt / len(probe)
+    n = int(max(len(probe), min(4096, budget_s / max(per_row, 1e-9))))
+    rows = sample_rows_uniform(wl.S, n, seed + 1)
+    dt, fl = oracle_sample(q, w, kc, wl, rows)
+    return {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "rows_per_s": len(rows) / dt,
+            "sample": f"{len(rows)} uniformly sampled query rows of batch 0 of the {wl.name} workload "
+                      f"(fp64 C oracle, OpenMP, {dt:.1f} s)"}
+
+
+def run_reference(args, world, rank, local):
+    """Reference arm: the CPU oracle as it stands on bounded row samples."""
+    from streaming_top_indexer_b200 import synth
+    if rank != 0:
+        return
+    wl = synth.WORKLOADS[args.workload]
+    dev = f"cuda:{local}" if torch.cuda.is_available() else "cpu"
+    q, w, kc = synth.generate(wl, seed=args.seed, device=dev)
+    from oracle import oracle as orc
+    cores = orc.max_threads()
+    probe = sample_rows_uniform(wl.S, max(cores, 8), args.seed)
+    dt, _ = oracle_sample(q, w, kc, wl, probe)
+    per_row = dt / len(probe)
+    steps_total = args.steps + args.warmup
+    n = int(max(8, min(1024, (args.ref_budget / steps_total) / max(per_row, 1e-9))))
+    for i in range(args.warmup):
+        oracle_sample(q, w, kc, wl, sample_rows_uniform(wl.S, n, args.seed + 100 + i))
+    tot_t, tot_f = 0.0, 0.0
+    for i in range(args.steps):
+        dt, fl = oracle_sample(q, w, kc, wl, sample_rows_uniform(wl.S, n, args.seed + 200 + i))
+        tot_t += dt
+        tot_f += fl
+    value = tot_f / tot_t / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot_t / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": config_of(wl, args),
+        "rows_per_s": n * args.steps / tot_t,
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{n} uniformly sampled query rows per step of the {wl.name} workload"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def config_of(wl, args):
+    return {"workload": wl.name, "B": wl.B, "S": wl.S, "T": wl.T, "H_I": wl.H, "d_I": wl.D, "m": wl.m,
+            "k": wl.k, "global_batch": wl.B * args.gpus, "seq_len": wl.S,
+            "parallelism": f"replicas{args.gpus}" if args.gpus > 1 else "single",
+            "l2": "inputs larger than L2 (q alone exceeds 126 MB); no flush between steps"}
+
+
+def run_ours(args, world, rank, local):
+    import streaming_top_indexer_b200 as si
+    from streaming_top_indexer_b200 import build as sbuild
+    from streaming_top_indexer_b200 import synth
+
+    if rank == 0 and sbuild.needs_build():
+        sbuild.build()
+    barrier(world)
+    dev = torch.device(f"cuda:{local}")
+    wl = synth.WORKLOADS[args.workload]
+    B, S, T, H, D, m, k = wl.B, wl.S, wl.T, wl.H, wl.D, wl.m, wl.k
+    torch.cuda.reset_peak_memory_stats(dev)
+    q, w, kc = synth.generate(wl, seed=args.seed + rank, device=dev)
+    idx = torch.empty((B, S, k), dtype=torch.int32, device=dev)
+    sc = torch.empty((B, S, k), dtype=torch.float32, device=dev)
+    ws_bytes = si.workspace_bytes(B, S, T, H, D, m, k)
+    ws = torch.zeros(ws_bytes, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        si.select_topk(q, w, kc, m, k, idx, sc, ws, stream)
+        si.sort_topk(idx, sc, stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    assert si.check_device_status(ws) == 0, "device error during warm-up"
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    sampler = ClockSampler(local)
+    with sampler:
+        barrier(world)
+        torch.cuda.synchronize(dev)
+        for i in range(args.steps):
+            ev[i][0].record(stream)
+            si.select_topk(q, w, kc, m, k, idx, sc, ws, stream)
+            ev[i][1].record(stream)
+            si.sort_topk(idx, sc, stream)
+            ev[i][2].record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(world)
+    assert si.check_device_status(ws) == 0, "device error during the timed region"
+    total_ms = ev[0][0].elapsed_time(ev[-1][2])
+    select_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    sort_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    peak_bytes = torch.cuda.max_memory_allocated(dev)
+    total_ms_max = all_max(total_ms, world, dev)
+
+    pairs = visible_pairs(B, S, T, m)
+    flops_rank = 2.0 * H * D * pairs
+    ms_per_step = total_ms_max / args.steps
+    value = world * flops_rank * args.steps / (total_ms_max * 1e-3) / 1e12
+    rows_per_s = world * B * S * args.steps / (total_ms_max * 1e-3)
+
+    peaks, peak_src = load_peaks()
+    sel_avg_ms = statistics.mean(select_ms)
+    achieved = flops_rank / (sel_avg_ms * 1e-3) / 1e12
+    traffic = ncu_traffic(wl.name)
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": achieved / peaks["bf16_tflops"], "traffic": traffic,
+                "peak_source": f"{peak_src} bf16 burst",
+                "frac_of_sustained": achieved / peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]),
+                "kernel": "select_kernel<64,128>" if (H, D) == (64, 128) else f"select_kernel<{H},{D}>",
+                "select_ms": sel_avg_ms, "sort_ms": statistics.mean(sort_ms)}
+
+    line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_of(wl, args),
+            "rows_per_s": rows_per_s, "peak_hbm_bytes": int(peak_bytes), "peak_hbm_gb": peak_bytes / 1e9,
+            "workspace_bytes": ws_bytes, "gpu_launches": 2 * args.steps, "roofline": roofline,
+            "clocks": sampler.summary()}
+
+    # end to end through the public API with host buffers
+    if not args.no_e2e:
+        line["e2e"] = e2e_measure(si, q, w, kc, wl, args, world, dev, stream, flops_rank)
+    del idx, sc
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(q, w, kc, wl, args.cpu_budget, args.seed)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def e2e_measure(si, q, w, kc, wl, args, world, dev, stream, flops_rank):
+    """Same metric through indexer_topk_host: pinned host inputs copied in,
+    outputs copied out, inside the timed region every step."""
+    qh = q.cpu().pin_memory()
+    wh = w.cpu().pin_memory()
+    kch = kc.cpu().pin_memory()
+    bufs = {}
+    steps = max(1, min(args.steps, args.e2e_steps))
+    for _ in range(2):
+        si.indexer_topk_host(qh, wh, kch, wl.m, wl.k, device=dev, buffers=bufs, stream=stream)
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    e0.record(stream)
+    for _ in range(steps):
+        si.indexer_topk_host(qh, wh, kch, wl.m, wl.k, device=dev, buffers=bufs, stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = all_max(e0.elapsed_time(e1), world, dev)
+    h2d = qh.numel() * 2 + wh.numel() * 4 + kch.numel() * 2
+    d2h = bufs["idx_h"].numel() * 4 + bufs["score_h"].numel() * 4
+    return {"value": world * flops_rank * steps / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": steps,
+            "ms_per_step": ms / steps}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="long")
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work")
+    ap.add_argument("--ref-budget", type=float, default=60.0, help="seconds of oracle work, reference arm")
+    args = ap.parse_args()
+    world, rank, local = dist_setup(args)
+    args.gpus = world if world > 1 else args.gpus
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank, local)
+        else:
+            run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,127 @@
+/*
+ * si.h -- C ABI of the streaming top-k indexer for NVIDIA B200 (sm_100a).
+ *
+ * The operation (StreamIndex: Memory-Bounded Compressed Sparse Attention via
+ * Streaming Top-k, arXiv 2605.02568v1, Abstract): the lightning indexer of
+ * Compressed Sparse Attention scores every compressed key for each query and
+ * keeps the top-k keys per query, without materialising the [B,S,H_I,T] fp32
+ * score tensor.  The Abstract names the score only "a learned scoring
+ * projection over compressed keys"; this library computes
+ *
+ *     score[b,t,s] = sum_h w[b,t,h] * max(0, sum_d q[b,t,h,d] * kc[b,s,d])
+ *
+ * over the keys visible to query t, key s being visible iff (s+1)*m <= t+1
+ * and s < T, i.e. s < V_t = min(T, floor((t+1)/m)).  Each output row holds
+ * min(k, V_t) keys ordered by score descending and, for equal scores, by key
+ * index ascending, followed by padding (index -1, score -infinity).
+ *
+ * Conventions for every entry point:
+ *  - All tensors are dense, contiguous and row-major, in device memory
+ *    unless stated otherwise.  q: bf16 [B,S,H_I,d_I]; w: fp32 [B,S,H_I];
+ *    kc: bf16 [B,T,d_I]; out_idx: int32 [B,S,k]; out_score: fp32 [B,S,k].
+ *  - q, w and kc must be 16-byte aligned; out_idx and out_score 4-byte
+ *    aligned.  The workspace must be 16-byte aligned.
+ *  - Supported: H_I in {8,16,32,64}; d_I in {64,128}; 1 <= k <= 2048;
+ *    m >= 1; B, S >= 1; T >= 0; S*H_I < 2^31; T < 2^31; B < 2^31.
+ *  - The caller owns every buffer; the library never allocates or frees
+ *    device memory.  Work is enqueued on `stream` (NULL = legacy default
+ *    stream) without any host synchronisation; results are ready when the
+ *    stream reaches that point.  Calls are reentrant; concurrent calls need
+ *    separate workspaces and outputs.  Results are deterministic.
+ *  - Argument errors are reported before anything is enqueued.  Errors of
+ *    the device (a bounded wait that expired) are recorded in the workspace
+ *    and read with si_check_device_status().
+ */
+#ifndef STREAMING_TOP_INDEXER_SI_H_
+#define STREAMING_TOP_INDEXER_SI_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SI_API __attribute__((visibility("default")))
+#else
+#define SI_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; declared here so callers need no CUDA header. */
+typedef struct CUstream_st* si_stream_t;
+
+typedef enum {
+    SI_OK = 0,
+    SI_ERR_INVALID_ARG = 1,        /* null pointer or out-of-range size */
+    SI_ERR_UNSUPPORTED = 2,        /* H_I, d_I or k outside the supported set */
+    SI_ERR_MISALIGNED = 3,         /* a pointer breaks the alignment rules */
+    SI_ERR_WORKSPACE_TOO_SMALL = 4,
+    SI_ERR_CUDA = 5,               /* a CUDA runtime/driver call failed */
+    SI_ERR_TIMEOUT = 6             /* a device-side wait expired (kernel aborted) */
+} si_status;
+
+/* Bytes of workspace si_indexer_topk needs for these sizes (host arithmetic
+ * only, no CUDA call).  At least 256.  It is O(number of SMs x top-k pool),
+ * independent of S and T, never O(S*T).  Returns 0 for unsupported sizes. */
+SI_API size_t si_workspace_bytes(int64_t B, int64_t S, int64_t T, int H_I, int d_I, int m, int k);
+
+/* The indexer step: top-k keys and scores of every query row.
+ * Enqueues: a 256-byte reset of the workspace header, the fused scoring and
+ * selection kernel, and the per-row sort.  Writes every element of out_idx
+ * and out_score, padding included. */
+SI_API si_status si_indexer_topk(const void* q, const float* w, const void* kc,
+                          int64_t B, int64_t S, int64_t T, int H_I, int d_I, int m, int k,
+                          int32_t* out_idx, float* out_score,
+                          void* workspace, size_t workspace_bytes, si_stream_t stream);
+
+/* First stage of si_indexer_topk alone: the fused scoring + selection kernel.
+ * Leaves each row's top-k set in out_idx/out_score unordered (padding at the
+ * tail).  Does not reset the workspace header.  Exposed so that the stages
+ * can be timed separately; si_indexer_topk == header reset + this + sort. */
+SI_API si_status si_select_topk(const void* q, const float* w, const void* kc,
+                         int64_t B, int64_t S, int64_t T, int H_I, int d_I, int m, int k,
+                         int32_t* out_idx, float* out_score,
+                         void* workspace, size_t workspace_bytes, si_stream_t stream);
+
+/* Second stage: orders each of the `rows` rows of k (index, score) pairs by
+ * score descending, then index ascending, padding last (in place). */
+SI_API si_status si_sort_topk(int32_t* out_idx, float* out_score, int64_t rows, int k,
+                       si_stream_t stream);
+
+/* The materialise path, for small problems: writes score[b,t,s] for every
+ * visible key into out_scores, fp32 [B,S,T] (entries of invisible keys are
+ * left untouched), through the same TMA + tcgen05 pipeline as the streaming
+ * path.  Same argument rules as si_indexer_topk; needs a workspace of at
+ * least 256 bytes. */
+SI_API si_status si_indexer_scores(const void* q, const float* w, const void* kc,
+                            int64_t B, int64_t S, int64_t T, int H_I, int d_I, int m,
+                            float* out_scores, void* workspace, size_t workspace_bytes,
+                            si_stream_t stream);
+
+/* Synchronises `stream`, then returns SI_OK or the device error recorded in
+ * the workspace header by the last call that used it (SI_ERR_TIMEOUT), or
+ * SI_ERR_CUDA if reading it failed. */
+SI_API si_status si_check_device_status(const void* workspace, si_stream_t stream);
+
+/* Self-test of the device-side bounded wait: launches a one-block kernel that
+ * waits on a barrier nobody arrives at, with a limit of limit_ns; the wait
+ * gives up and records SI_ERR_TIMEOUT in the workspace header, which
+ * si_check_device_status() then returns.  No fault, trap or hang. */
+SI_API si_status si_selftest_timeout(void* workspace, size_t workspace_bytes, uint64_t limit_ns,
+                              si_stream_t stream);
+
+/* Device-side wait limit, in nanoseconds, used by later calls (default 2 s). */
+SI_API void si_set_timeout_ns(uint64_t ns);
+
+/* Human-readable name of a status code. */
+SI_API const char* si_status_string(si_status s);
+
+/* Library version string. */
+SI_API const char* si_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* STREAMING_TOP_INDEXER_SI_H_ */

@@ -1,0 +1,244 @@
+"""Streaming top-k indexer (CSA indexer step) for NVIDIA B200, sm_100a.
+
+Thin Python binding of the C ABI in ``include/si.h`` (``lib/libsi.so``):
+argument marshalling only.  Every step of the computation runs in the
+library's CUDA kernels; there is no CPU fallback, and every call raises if
+the library is missing or a tensor is not a CUDA tensor of the right dtype.
+
+The operation (StreamIndex: Memory-Bounded Compressed Sparse Attention via
+Streaming Top-k, Abstract): for each query row t, score every compressed
+key s it can see, ``score = sum_h w[t,h] * ReLU(q[t,h,:] . kc[s,:])`` with s
+visible iff (s+1)*m <= t+1, and return the top-k keys (score descending,
+equal scores to the lower index, padding index -1 / score -inf) without
+materialising the [B,S,H_I,T] score tensor.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "SIError", "library_path", "load_library", "workspace_bytes", "indexer_topk",
+    "select_topk", "sort_topk", "indexer_scores", "check_device_status",
+    "selftest_timeout", "set_timeout_ns", "indexer_topk_host", "version",
+]
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_PKG, "lib", "libsi.so")
+_lib = None
+
+SI_STATUS = {0: "SI_OK", 1: "SI_ERR_INVALID_ARG", 2: "SI_ERR_UNSUPPORTED", 3: "SI_ERR_MISALIGNED",
+             4: "SI_ERR_WORKSPACE_TOO_SMALL", 5: "SI_ERR_CUDA", 6: "SI_ERR_TIMEOUT"}
+
+
+class SIError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {SI_STATUS.get(status, status)}")
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def _declare(lib):
+    c = ctypes
+    vp, i64, i32, sz = c.c_void_p, c.c_int64, c.c_int, c.c_size_t
+    lib.si_workspace_bytes.restype = sz
+    lib.si_workspace_bytes.argtypes = [i64, i64, i64, i32, i32, i32, i32]
+    topk_args = [vp, vp, vp, i64, i64, i64, i32, i32, i32, i32, vp, vp, vp, sz, vp]
+    for name in ("si_indexer_topk", "si_select_topk"):
+        fn = getattr(lib, name)
+        fn.restype = c.c_int
+        fn.argtypes = topk_args
+    lib.si_sort_topk.restype = c.c_int
+    lib.si_sort_topk.argtypes = [vp, vp, i64, i32, vp]
+    lib.si_indexer_scores.restype = c.c_int
+    lib.si_indexer_scores.argtypes = [vp, vp, vp, i64, i64, i64, i32, i32, i32, vp, vp, sz, vp]
+    lib.si_check_device_status.restype = c.c_int
+    lib.si_check_device_status.argtypes = [vp, vp]
+    lib.si_selftest_timeout.restype = c.c_int
+    lib.si_selftest_timeout.argtypes = [vp, sz, c.c_uint64, vp]
+    lib.si_set_timeout_ns.restype = None
+    lib.si_set_timeout_ns.argtypes = [c.c_uint64]
+    lib.si_status_string.restype = c.c_char_p
+    lib.si_status_string.argtypes = [c.c_int]
+    lib.si_version.restype = c.c_char_p
+    lib.si_version.argtypes = []
+    return lib
+
+
+def load_library():
+    """Load lib/libsi.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError(
+                f"{_LIB_PATH} is missing: build it with `python -m streaming_top_indexer_b200.build`")
+        _lib = _declare(ctypes.CDLL(_LIB_PATH))
+    return _lib
+
+
+def version() -> str:
+    return load_library().si_version().decode()
+
+
+def set_timeout_ns(ns: int) -> None:
+    load_library().si_set_timeout_ns(int(ns))
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _need(t: torch.Tensor, name: str, dtype, ndim: int):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != ndim or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous {ndim}-d tensor")
+
+
+def _check(rc: int, what: str):
+    if rc != 0:
+        raise SIError(rc, what)
+
+
+def _dims(q, w, kc):
+    _need(q, "q", torch.bfloat16, 4)
+    _need(w, "w", torch.float32, 3)
+    _need(kc, "kc", torch.bfloat16, 3)
+    B, S, H, D = q.shape
+    if tuple(w.shape) != (B, S, H) or kc.shape[0] != B or kc.shape[2] != D:
+        raise ValueError(f"shape mismatch: q {tuple(q.shape)} w {tuple(w.shape)} kc {tuple(kc.shape)}")
+    return B, S, kc.shape[1], H, D
+
+
+def workspace_bytes(B: int, S: int, T: int, H: int, D: int, m: int, k: int) -> int:
+    n = load_library().si_workspace_bytes(B, S, T, H, D, m, k)
+    if n == 0:
+        raise SIError(2, "si_workspace_bytes")
+    return int(n)
+
+
+def _outputs(B, S, k, device, out_idx, out_score):
+    if out_idx is None:
+        out_idx = torch.empty((B, S, k), dtype=torch.int32, device=device)
+    if out_score is None:
+        out_score = torch.empty((B, S, k), dtype=torch.float32, device=device)
+    _need(out_idx, "out_idx", torch.int32, 3)
+    _need(out_score, "out_score", torch.float32, 3)
+    if tuple(out_idx.shape) != (B, S, k) or tuple(out_score.shape) != (B, S, k):
+        raise ValueError("outputs must be [B,S,k]")
+    return out_idx, out_score
+
+
+def _workspace(B, S, T, H, D, m, k, device, workspace):
+    need = workspace_bytes(B, S, T, H, D, m, k)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=device)
+    if not workspace.is_cuda or workspace.dtype != torch.uint8:
+        raise ValueError("workspace must be a CUDA uint8 tensor")
+    return workspace
+
+
+def _topk_call(fn_name, q, w, kc, m, k, out_idx, out_score, workspace, stream):
+    B, S, T, H, D = _dims(q, w, kc)
+    out_idx, out_score = _outputs(B, S, k, q.device, out_idx, out_score)
+    workspace = _workspace(B, S, T, H, D, m, k, q.device, workspace)
+    fn = getattr(load_library(), fn_name)
+    _check(fn(q.data_ptr(), w.data_ptr(), kc.data_ptr() if T > 0 else None, B, S, T, H, D, m, k,
+              out_idx.data_ptr(), out_score.data_ptr(), workspace.data_ptr(), workspace.numel(),
+              _stream(stream)), fn_name)
+    return out_idx, out_score
+
+
+def indexer_topk(q, w, kc, m: int, k: int, out_idx=None, out_score=None, workspace=None, stream=None):
+    """Top-k keys and scores of every query row (si_indexer_topk).
+
+    q bf16 [B,S,H_I,d_I], w fp32 [B,S,H_I], kc bf16 [B,T,d_I] on the GPU.
+    Returns (idx int32 [B,S,k], score fp32 [B,S,k]), asynchronously on
+    ``stream`` (default: torch's current stream).
+    """
+    return _topk_call("si_indexer_topk", q, w, kc, m, k, out_idx, out_score, workspace, stream)
+
+
+def select_topk(q, w, kc, m: int, k: int, out_idx=None, out_score=None, workspace=None, stream=None):
+    """First stage only (si_select_topk): each row's top-k set, unordered."""
+    return _topk_call("si_select_topk", q, w, kc, m, k, out_idx, out_score, workspace, stream)
+
+
+def sort_topk(out_idx, out_score, stream=None):
+    """Second stage only (si_sort_topk): order rows in place."""
+    _need(out_idx, "out_idx", torch.int32, 3)
+    _need(out_score, "out_score", torch.float32, 3)
+    B, S, k = out_idx.shape
+    _check(load_library().si_sort_topk(out_idx.data_ptr(), out_score.data_ptr(), B * S, k, _stream(stream)),
+           "si_sort_topk")
+    return out_idx, out_score
+
+
+def indexer_scores(q, w, kc, m: int, out=None, workspace=None, stream=None):
+    """Materialise path for small problems (si_indexer_scores): dense fp32
+    [B,S,T] scores; entries of keys a row cannot see are left as given in
+    ``out`` (default: NaN)."""
+    B, S, T, H, D = _dims(q, w, kc)
+    if out is None:
+        out = torch.full((B, S, T), float("nan"), dtype=torch.float32, device=q.device)
+    _need(out, "out", torch.float32, 3)
+    if workspace is None:
+        workspace = torch.empty(256, dtype=torch.uint8, device=q.device)
+    _check(load_library().si_indexer_scores(q.data_ptr(), w.data_ptr(), kc.data_ptr() if T > 0 else None,
+                                            B, S, T, H, D, m, out.data_ptr(), workspace.data_ptr(),
+                                            workspace.numel(), _stream(stream)), "si_indexer_scores")
+    return out
+
+
+def check_device_status(workspace, stream=None) -> int:
+    """Synchronise and return the device status word of the last call (0 = OK)."""
+    return int(load_library().si_check_device_status(workspace.data_ptr(), _stream(stream)))
+
+
+def selftest_timeout(workspace, limit_ns: int, stream=None) -> int:
+    """Run the bounded-wait self-test; returns the device status it left."""
+    _check(load_library().si_selftest_timeout(workspace.data_ptr(), workspace.numel(), int(limit_ns),
+                                              _stream(stream)), "si_selftest_timeout")
+    return check_device_status(workspace, stream)
+
+
+def indexer_topk_host(q, w, kc, m: int, k: int, device="cuda", buffers=None, stream=None):
+    """End-to-end call on host tensors: copies q, w, kc to the GPU, runs
+    si_indexer_topk and copies (idx, score) back into host tensors.
+
+    ``buffers`` may hold preallocated device tensors ("q","w","kc","idx",
+    "score","ws") and pinned host outputs ("idx_h","score_h") to reuse.
+    Returns (idx_h, score_h); the copies are asynchronous on ``stream`` and
+    complete when the stream is synchronised.
+    """
+    b = {} if buffers is None else buffers
+    dev = torch.device(device)
+    B, S, H, D = q.shape
+    T = kc.shape[1]
+    if "q" not in b:
+        b["q"] = torch.empty(q.shape, dtype=torch.bfloat16, device=dev)
+        b["w"] = torch.empty(w.shape, dtype=torch.float32, device=dev)
+        b["kc"] = torch.empty(kc.shape, dtype=torch.bfloat16, device=dev)
+        b["idx"] = torch.empty((B, S, k), dtype=torch.int32, device=dev)
+        b["score"] = torch.empty((B, S, k), dtype=torch.float32, device=dev)
+        b["ws"] = torch.empty(workspace_bytes(B, S, T, H, D, m, k), dtype=torch.uint8, device=dev)
+        b["idx_h"] = torch.empty((B, S, k), dtype=torch.int32, pin_memory=True)
+        b["score_h"] = torch.empty((B, S, k), dtype=torch.float32, pin_memory=True)
+    s = stream if stream is not None else torch.cuda.current_stream(dev)
+    with torch.cuda.stream(s):
+        b["q"].copy_(q, non_blocking=True)
+        b["w"].copy_(w, non_blocking=True)
+        b["kc"].copy_(kc, non_blocking=True)
+        indexer_topk(b["q"], b["w"], b["kc"], m, k, b["idx"], b["score"], b["ws"], s)
+        b["idx_h"].copy_(b["idx"], non_blocking=True)
+        b["score_h"].copy_(b["score"], non_blocking=True)
+    return b["idx_h"], b["score_h"]

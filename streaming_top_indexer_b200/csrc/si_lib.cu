@@ -1,0 +1,316 @@
+// si_lib.cu -- host side of the C ABI (include/si.h): argument checks,
+// workspace sizing, TMA descriptors and kernel launches on the caller's
+// stream.  No allocation, no host synchronisation (except in
+// si_check_device_status, which is documented to synchronise).
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "si.h"
+#include "si_ptx.cuh"
+#include "si_keys.cuh"
+#include "si_select.cuh"
+#include "si_sort.cuh"
+
+namespace {
+
+constexpr int kMaxCtas = 148;                 // persistent CTAs (one per B200 SM)
+constexpr size_t kHeaderBytes = 256;          // error word + reserved
+constexpr uint32_t kMaxDynSmem = 232448;      // 227 KB opt-in per block on sm_100
+constexpr uint32_t kMinDynSmem = 120 * 1024;  // > half an SM: one CTA per SM, so
+                                              // two CTAs never compete for TMEM
+std::atomic<uint64_t> g_timeout_ns{2000000000ull};
+
+bool supported_h(int h) { return h == 8 || h == 16 || h == 32 || h == 64; }
+bool supported_d(int d) { return d == 64 || d == 128; }
+
+int pool_capacity(int k) {
+    int p = 2 * k > k + 256 ? 2 * k : k + 256;
+    return (p + 31) / 32 * 32;
+}
+
+// Shared-memory bytes of the select kernel without / with the pools in smem.
+uint32_t select_smem(int H, int D, bool pool_in_smem, int P) {
+#define SI_CASE(HH, DD) \
+    if (H == HH && D == DD) return si::SelCfg<HH, DD>::smem_bytes(pool_in_smem, P);
+    SI_CASE(8, 64) SI_CASE(8, 128) SI_CASE(16, 64) SI_CASE(16, 128)
+    SI_CASE(32, 64) SI_CASE(32, 128) SI_CASE(64, 64) SI_CASE(64, 128)
+#undef SI_CASE
+    return 0;
+}
+
+bool pool_fits_smem(int H, int D, int k) { return select_smem(H, D, true, pool_capacity(k)) <= kMaxDynSmem; }
+
+size_t global_pool_bytes(int H, int D, int k) {
+    if (pool_fits_smem(H, D, k)) return 0;
+    const size_t QT = 256 / H;
+    return static_cast<size_t>(kMaxCtas) * QT * pool_capacity(k) * sizeof(uint64_t);
+}
+
+si_status check_common(const void* q, const float* w, const void* kc, int64_t B, int64_t S, int64_t T,
+                       int H, int D, int m) {
+    if (B < 1 || S < 1 || T < 0 || m < 1) return SI_ERR_INVALID_ARG;
+    if (!q || !w || (T > 0 && !kc)) return SI_ERR_INVALID_ARG;
+    if (!supported_h(H) || !supported_d(D)) return SI_ERR_UNSUPPORTED;
+    if (S * H >= (int64_t{1} << 31) || T >= (int64_t{1} << 31) || B >= (int64_t{1} << 31))
+        return SI_ERR_UNSUPPORTED;
+    auto a16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
+    if (!a16(q) || !a16(w) || (T > 0 && !a16(kc))) return SI_ERR_MISALIGNED;
+    return SI_OK;
+}
+
+si_status check_topk(const void* q, const float* w, const void* kc, int64_t B, int64_t S, int64_t T, int H,
+                     int D, int m, int k, const int32_t* out_idx, const float* out_score, const void* ws,
+                     size_t ws_bytes) {
+    si_status st = check_common(q, w, kc, B, S, T, H, D, m);
+    if (st != SI_OK) return st;
+    if (k < 1 || k > 2048) return SI_ERR_UNSUPPORTED;
+    if (!out_idx || !out_score || !ws) return SI_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(out_idx) & 3u) || (reinterpret_cast<uintptr_t>(out_score) & 3u) ||
+        (reinterpret_cast<uintptr_t>(ws) & 15u))
+        return SI_ERR_MISALIGNED;
+    if (ws_bytes < si_workspace_bytes(B, S, T, H, D, m, k)) return SI_ERR_WORKSPACE_TOO_SMALL;
+    return SI_OK;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+bool encode_3d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t d0, uint64_t d1,
+               uint64_t d2, uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t box0, uint32_t box1,
+               CUtensorMapSwizzle sw) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {d0, d1, d2};
+    cuuint64_t strides[2] = {stride1_bytes, stride2_bytes};
+    cuuint32_t box[3] = {box0, box1, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    std::memset(map, 0, sizeof(*map));
+    CUresult r = enc(map, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+struct DeviceInfo {
+    int sms = 0;
+    bool attr_set[2][4][2] = {};  // [D==128][log2(H/8)][unused]
+};
+
+std::mutex g_dev_mu;
+DeviceInfo g_dev[64];
+
+int device_sms(int dev) {
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    if (dev < 0 || dev >= 64) return 0;
+    if (g_dev[dev].sms == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+        g_dev[dev].sms = n;
+    }
+    return g_dev[dev].sms;
+}
+
+template <int H, int D>
+si_status launch_select_t(const void* q, const float* w, const void* kc, int64_t B, int64_t S, int64_t T, int m,
+                          int k, int32_t* out_idx, float* out_score, float* dense, void* ws, cudaStream_t stream) {
+    using C = si::SelCfg<H, D>;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return SI_ERR_CUDA;
+    const int sms = device_sms(dev);
+    if (sms <= 0) return SI_ERR_CUDA;
+
+    si::SelectParams p{};
+    p.B = B;
+    p.S = S;
+    p.T = T;
+    p.m = m;
+    p.k = dense ? 1 : k;
+    p.P = pool_capacity(p.k);
+    p.nblk = (S + C::QT - 1) / C::QT;
+    p.units = B * p.nblk;
+    p.out_idx = out_idx;
+    p.out_score = out_score;
+    p.dense = dense;
+    p.err = static_cast<uint32_t*>(ws);
+    p.timeout_ns = g_timeout_ns.load();
+    const bool smem_pool = dense || pool_fits_smem(H, D, p.k);
+    p.gpool = smem_pool ? nullptr
+                        : reinterpret_cast<uint64_t*>(static_cast<uint8_t*>(ws) + kHeaderBytes);
+
+    CUtensorMap tq, tkc, tw;
+    const uint64_t bf = 2;
+    if (!encode_3d(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q, D, static_cast<uint64_t>(S) * H, B, D * bf,
+                   static_cast<uint64_t>(S) * H * D * bf, 64, C::N, CU_TENSOR_MAP_SWIZZLE_128B))
+        return SI_ERR_CUDA;
+    if (!encode_3d(&tkc, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kc, D, T, B, D * bf, static_cast<uint64_t>(T) * D * bf,
+                   64, C::BM, CU_TENSOR_MAP_SWIZZLE_128B))
+        return SI_ERR_CUDA;
+    if (!encode_3d(&tw, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, w, H, S, B, H * 4ull, static_cast<uint64_t>(S) * H * 4ull,
+                   H, C::QT, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return SI_ERR_CUDA;
+
+    uint32_t smem = C::smem_bytes(smem_pool, p.P);
+    if (smem < kMinDynSmem) smem = kMinDynSmem;
+    if (smem > kMaxDynSmem) return SI_ERR_UNSUPPORTED;
+    auto kern = si::select_kernel<H, D>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
+        cudaSuccess)
+        return SI_ERR_CUDA;
+    int64_t grid = sms < kMaxCtas ? sms : kMaxCtas;
+    if (grid > p.units) grid = p.units;
+    kern<<<static_cast<unsigned>(grid), C::THREADS, smem, stream>>>(tq, tkc, tw, p);
+    return cudaGetLastError() == cudaSuccess ? SI_OK : SI_ERR_CUDA;
+}
+
+si_status launch_select(const void* q, const float* w, const void* kc, int64_t B, int64_t S, int64_t T, int H, int D,
+                        int m, int k, int32_t* out_idx, float* out_score, float* dense, void* ws,
+                        cudaStream_t stream) {
+#define SI_CASE(HH, DD)     \
+    if (H == HH && D == DD) \
+        return launch_select_t<HH, DD>(q, w, kc, B, S, T, m, k, out_idx, out_score, dense, ws, stream);
+    SI_CASE(8, 64) SI_CASE(8, 128) SI_CASE(16, 64) SI_CASE(16, 128)
+    SI_CASE(32, 64) SI_CASE(32, 128) SI_CASE(64, 64) SI_CASE(64, 128)
+#undef SI_CASE
+    return SI_ERR_UNSUPPORTED;
+}
+
+si_status launch_pad(int32_t* out_idx, float* out_score, int64_t n, cudaStream_t stream) {
+    if (n <= 0) return SI_OK;
+    int64_t blocks = (n + 255) / 256;
+    if (blocks > 4096) blocks = 4096;
+    si::pad_rows_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(out_idx, out_score, n);
+    return cudaGetLastError() == cudaSuccess ? SI_OK : SI_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t si_workspace_bytes(int64_t B, int64_t S, int64_t T, int H_I, int d_I, int m, int k) {
+    if (B < 1 || S < 1 || T < 0 || m < 1 || k < 1 || k > 2048 || !supported_h(H_I) || !supported_d(d_I)) return 0;
+    return kHeaderBytes + global_pool_bytes(H_I, d_I, k);
+}
+
+si_status si_select_topk(const void* q, const float* w, const void* kc, int64_t B, int64_t S, int64_t T, int H_I,
+                         int d_I, int m, int k, int32_t* out_idx, float* out_score, void* workspace,
+                         size_t workspace_bytes, si_stream_t stream) {
+    si_status st = check_topk(q, w, kc, B, S, T, H_I, d_I, m, k, out_idx, out_score, workspace, workspace_bytes);
+    if (st != SI_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (T == 0) return launch_pad(out_idx, out_score, B * S * k, s);
+    return launch_select(q, w, kc, B, S, T, H_I, d_I, m, k, out_idx, out_score, nullptr, workspace, s);
+}
+
+si_status si_sort_topk(int32_t* out_idx, float* out_score, int64_t rows, int k, si_stream_t stream) {
+    if (!out_idx || !out_score || rows < 0) return SI_ERR_INVALID_ARG;
+    if (k < 1 || k > 2048) return SI_ERR_UNSUPPORTED;
+    if ((reinterpret_cast<uintptr_t>(out_idx) & 3u) || (reinterpret_cast<uintptr_t>(out_score) & 3u))
+        return SI_ERR_MISALIGNED;
+    if (rows == 0) return SI_OK;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const int64_t blocks64 = (rows + si::kSortWarps - 1) / si::kSortWarps;
+    if (blocks64 > 0x7FFFFFFF) return SI_ERR_UNSUPPORTED;
+    const unsigned blocks = static_cast<unsigned>(blocks64);
+    const unsigned threads = 32 * si::kSortWarps;
+    int k2 = 32;
+    while (k2 < k) k2 <<= 1;
+    switch (k2 / 32) {
+        case 1: si::sort_rows_kernel<1><<<blocks, threads, 0, s>>>(out_idx, out_score, rows, k); break;
+        case 2: si::sort_rows_kernel<2><<<blocks, threads, 0, s>>>(out_idx, out_score, rows, k); break;
+        case 4: si::sort_rows_kernel<4><<<blocks, threads, 0, s>>>(out_idx, out_score, rows, k); break;
+        case 8: si::sort_rows_kernel<8><<<blocks, threads, 0, s>>>(out_idx, out_score, rows, k); break;
+        case 16: si::sort_rows_kernel<16><<<blocks, threads, 0, s>>>(out_idx, out_score, rows, k); break;
+        case 32: si::sort_rows_kernel<32><<<blocks, threads, 0, s>>>(out_idx, out_score, rows, k); break;
+        case 64: si::sort_rows_kernel<64><<<blocks, threads, 0, s>>>(out_idx, out_score, rows, k); break;
+        default: return SI_ERR_UNSUPPORTED;
+    }
+    return cudaGetLastError() == cudaSuccess ? SI_OK : SI_ERR_CUDA;
+}
+
+si_status si_indexer_topk(const void* q, const float* w, const void* kc, int64_t B, int64_t S, int64_t T, int H_I,
+                          int d_I, int m, int k, int32_t* out_idx, float* out_score, void* workspace,
+                          size_t workspace_bytes, si_stream_t stream) {
+    si_status st = check_topk(q, w, kc, B, S, T, H_I, d_I, m, k, out_idx, out_score, workspace, workspace_bytes);
+    if (st != SI_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(workspace, 0, kHeaderBytes, s) != cudaSuccess) return SI_ERR_CUDA;
+    if (T == 0) return launch_pad(out_idx, out_score, B * S * k, s);
+    st = launch_select(q, w, kc, B, S, T, H_I, d_I, m, k, out_idx, out_score, nullptr, workspace, s);
+    if (st != SI_OK) return st;
+    return si_sort_topk(out_idx, out_score, B * S, k, stream);
+}
+
+si_status si_indexer_scores(const void* q, const float* w, const void* kc, int64_t B, int64_t S, int64_t T, int H_I,
+                            int d_I, int m, float* out_scores, void* workspace, size_t workspace_bytes,
+                            si_stream_t stream) {
+    si_status st = check_common(q, w, kc, B, S, T, H_I, d_I, m);
+    if (st != SI_OK) return st;
+    if (!out_scores || !workspace) return SI_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(out_scores) & 3u) || (reinterpret_cast<uintptr_t>(workspace) & 15u))
+        return SI_ERR_MISALIGNED;
+    if (workspace_bytes < kHeaderBytes) return SI_ERR_WORKSPACE_TOO_SMALL;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(workspace, 0, kHeaderBytes, s) != cudaSuccess) return SI_ERR_CUDA;
+    if (T == 0) return SI_OK;
+    return launch_select(q, w, kc, B, S, T, H_I, d_I, m, 1, nullptr, nullptr, out_scores, workspace, s);
+}
+
+si_status si_check_device_status(const void* workspace, si_stream_t stream) {
+    if (!workspace) return SI_ERR_INVALID_ARG;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint32_t word = 0;
+    if (cudaMemcpyAsync(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return SI_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return SI_ERR_CUDA;
+    if (word == 0) return SI_OK;
+    if (word == si::kErrTimeout) return SI_ERR_TIMEOUT;
+    return SI_ERR_CUDA;
+}
+
+si_status si_selftest_timeout(void* workspace, size_t workspace_bytes, uint64_t limit_ns, si_stream_t stream) {
+    if (!workspace) return SI_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(workspace) & 15u) return SI_ERR_MISALIGNED;
+    if (workspace_bytes < kHeaderBytes) return SI_ERR_WORKSPACE_TOO_SMALL;
+    if (limit_ns == 0 || limit_ns > 10000000000ull) return SI_ERR_INVALID_ARG;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(workspace, 0, kHeaderBytes, s) != cudaSuccess) return SI_ERR_CUDA;
+    si::timeout_selftest_kernel<<<1, 32, 0, s>>>(static_cast<uint32_t*>(workspace), limit_ns);
+    return cudaGetLastError() == cudaSuccess ? SI_OK : SI_ERR_CUDA;
+}
+
+void si_set_timeout_ns(uint64_t ns) {
+    if (ns > 0) g_timeout_ns.store(ns);
+}
+
+const char* si_status_string(si_status s) {
+    switch (s) {
+        case SI_OK: return "SI_OK";
+        case SI_ERR_INVALID_ARG: return "SI_ERR_INVALID_ARG";
+        case SI_ERR_UNSUPPORTED: return "SI_ERR_UNSUPPORTED";
+        case SI_ERR_MISALIGNED: return "SI_ERR_MISALIGNED";
+        case SI_ERR_WORKSPACE_TOO_SMALL: return "SI_ERR_WORKSPACE_TOO_SMALL";
+        case SI_ERR_CUDA: return "SI_ERR_CUDA";
+        case SI_ERR_TIMEOUT: return "SI_ERR_TIMEOUT";
+    }
+    return "SI_ERR_UNKNOWN";
+}
+
+const char* si_version(void) { return "streaming_top_indexer_b200 0.1.0 (sm_100a)"; }
+
+}  // extern "C"

@@ -1,0 +1,95 @@
+"""The C-ABI library without a GPU: it loads, exports every function the
+header declares, sizes workspaces on the host and rejects bad arguments
+before touching CUDA."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import streaming_top_indexer_b200 as si
+from streaming_top_indexer_b200 import build as sbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "si.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    sbuild.build()
+    return si.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(si_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for need in ("si_workspace_bytes", "si_indexer_topk", "si_check_device_status", "si_status_string"):
+        assert need in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    raw = ctypes.CDLL(si.library_path())
+    for name in declared_functions():
+        assert hasattr(raw, name), f"{name} not exported"
+
+
+def test_only_declared_symbols_are_exported():
+    out = os.popen(f"nm -D --defined-only {si.library_path()}").read()
+    exported = sorted(set(re.findall(r" T (si_\w+)", out)))
+    assert exported == declared_functions()
+
+
+def test_status_strings(lib):
+    for code, name in si.SI_STATUS.items():
+        assert lib.si_status_string(code).decode() == name
+
+
+def test_workspace_bytes_host_arithmetic(lib):
+    # pools fit in shared memory: header only
+    assert si.workspace_bytes(1, 262144, 65536, 64, 128, 4, 512) == 256
+    assert si.workspace_bytes(1, 2048, 512, 8, 64, 4, 64) == 256
+    # k = 2048 at H_I=64: 148 CTAs x 4 queries x 4096-entry pools x 8 bytes
+    assert si.workspace_bytes(4, 131072, 32768, 64, 128, 4, 2048) == 256 + 148 * 4 * 4096 * 8
+    # independent of S and T (never O(S*T))
+    assert si.workspace_bytes(1, 1 << 20, 1 << 18, 64, 128, 4, 2048) == si.workspace_bytes(1, 64, 16, 64, 128, 4, 2048)
+    for bad in [(1, 10, 4, 12, 128, 4, 8), (1, 10, 4, 64, 96, 4, 8), (1, 10, 4, 64, 128, 4, 0),
+                (1, 10, 4, 64, 128, 4, 4096), (0, 10, 4, 64, 128, 4, 8), (1, 10, 4, 64, 128, 0, 8)]:
+        assert lib.si_workspace_bytes(*bad) == 0
+
+
+def call_topk(lib, q=16, w=16, kc=16, B=1, S=8, T=2, H=64, D=128, m=4, k=4, oi=16, os_=16, ws=16, wsb=1 << 20):
+    return lib.si_indexer_topk(q, w, kc, B, S, T, H, D, m, k, oi, os_, ws, wsb, None)
+
+
+def test_argument_errors_before_any_cuda_call(lib):
+    assert call_topk(lib, q=0) == 1          # null q
+    assert call_topk(lib, oi=0) == 1         # null output
+    assert call_topk(lib, ws=0) == 1         # null workspace
+    assert call_topk(lib, B=0) == 1
+    assert call_topk(lib, m=0) == 1
+    assert call_topk(lib, H=12) == 2         # unsupported H_I
+    assert call_topk(lib, D=96) == 2         # unsupported d_I
+    assert call_topk(lib, k=4096) == 2       # k too large
+    assert call_topk(lib, S=1 << 26) == 2    # S*H_I >= 2^31
+    assert call_topk(lib, q=24) == 3         # q not 16-byte aligned
+    assert call_topk(lib, kc=8) == 3
+    assert call_topk(lib, oi=18) == 3        # out_idx not 4-byte aligned
+    assert call_topk(lib, wsb=16) == 4       # workspace too small
+    assert lib.si_sort_topk(16, 16, 4, 0, None) == 2
+    assert lib.si_sort_topk(0, 16, 4, 8, None) == 1
+    assert lib.si_indexer_scores(16, 16, 16, 1, 8, 2, 64, 128, 4, 16, 16, 8, None) == 4
+    assert lib.si_selftest_timeout(0, 256, 1000, None) == 1
+
+
+def test_python_binding_refuses_cpu_tensors():
+    import torch
+    q = torch.zeros((1, 8, 64, 128), dtype=torch.bfloat16)
+    w = torch.zeros((1, 8, 64))
+    kc = torch.zeros((1, 2, 128), dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        si.indexer_topk(q, w, kc, 4, 4)
