@@ -16,6 +16,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB_DIR = os.path.join(PKG, "lib")
 LIB_PATH = os.path.join(LIB_DIR, "libsi.so")
+TRACE_LIB_PATH = os.path.join(LIB_DIR, "libsi_trace.so")  # cycle-tracing build (SI_TRACE)
 SOURCES = [os.path.join(CSRC, "si_lib.cu")]
 HEADERS = [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith(".cuh")] + [
     os.path.join(INCLUDE, "si.h")]
@@ -43,11 +44,14 @@ def needs_build() -> bool:
     return any(os.path.getmtime(f) > t for f in SOURCES + HEADERS)
 
 
-def build(force: bool = False, verbose: bool = False, extra=()) -> str:
-    if not force and not needs_build():
+def build(force: bool = False, verbose: bool = False, extra=(), trace: bool = False) -> str:
+    out = TRACE_LIB_PATH if trace else LIB_PATH
+    if not trace and not force and not needs_build():
         return LIB_PATH
     os.makedirs(LIB_DIR, exist_ok=True)
-    tmp = LIB_PATH + ".tmp"
+    tmp = out + ".tmp"
+    if trace:
+        extra = [*extra, "-DSI_TRACE"]
     cmd = [nvcc(), *NVCC_FLAGS, *extra, "-I", INCLUDE, "-I", CSRC, "-shared", *SOURCES, "-o", tmp,
            "-Xlinker", "-rpath,/usr/local/cuda/lib64"]
     if verbose:
@@ -57,10 +61,10 @@ def build(force: bool = False, verbose: bool = False, extra=()) -> str:
         raise RuntimeError(f"nvcc failed ({res.returncode}):\n{res.stderr[-8000:]}")
     if verbose and res.stderr:
         print(res.stderr, file=sys.stderr)
-    os.replace(tmp, LIB_PATH)
-    return LIB_PATH
+    os.replace(tmp, out)
+    return out
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose=True,
+    print(build(force="--force" in sys.argv, verbose=True, trace="--trace" in sys.argv,
                 extra=["-Xptxas", "-v"] if "--ptxas-v" in sys.argv else []))

@@ -29,12 +29,7 @@ std::atomic<uint64_t> g_timeout_ns{2000000000ull};
 bool supported_h(int h) { return h == 8 || h == 16 || h == 32 || h == 64; }
 bool supported_d(int d) { return d == 64 || d == 128; }
 
-int pool_capacity(int k) {
-    int p = 2 * k > k + 256 ? 2 * k : k + 256;
-    return (p + 31) / 32 * 32;
-}
-
-// Shared-memory bytes of the select kernel without / with the pools in smem.
+// Shared-memory bytes (dynamic + static) of the select kernel.
 uint32_t select_smem(int H, int D, bool pool_in_smem, int P) {
 #define SI_CASE(HH, DD) \
     if (H == HH && D == DD) return si::SelCfg<HH, DD>::smem_bytes(pool_in_smem, P);
@@ -44,12 +39,32 @@ uint32_t select_smem(int H, int D, bool pool_in_smem, int P) {
     return 0;
 }
 
-bool pool_fits_smem(int H, int D, int k) { return select_smem(H, D, true, pool_capacity(k)) <= kMaxDynSmem; }
+// Where the per-query candidate pools live and how large they are.  A pool
+// holds at least max(2k, k+256) entries; in shared memory it takes all the
+// room left (fewer pool cuts), otherwise 4k entries in the workspace.
+struct PoolPlan {
+    bool smem;
+    int P;
+};
+
+PoolPlan pool_plan(int H, int D, int k) {
+    auto r32 = [](int x) { return (x + 31) / 32 * 32; };
+    const int min_p = r32(2 * k > k + 256 ? 2 * k : k + 256);
+    const uint32_t qt = 256u / static_cast<uint32_t>(H);
+    const uint32_t fixed = select_smem(H, D, false, 0);
+    if (fixed + qt * static_cast<uint32_t>(min_p) * 8u <= kMaxDynSmem) {
+        int p = static_cast<int>((kMaxDynSmem - fixed) / (qt * 8u)) / 32 * 32;
+        if (p > 65504) p = 65504;  // pool counts are 16-bit fields
+        return {true, p};
+    }
+    return {false, r32(4 * k > k + 256 ? 4 * k : k + 256)};
+}
 
 size_t global_pool_bytes(int H, int D, int k) {
-    if (pool_fits_smem(H, D, k)) return 0;
+    const PoolPlan pp = pool_plan(H, D, k);
+    if (pp.smem) return 0;
     const size_t QT = 256 / H;
-    return static_cast<size_t>(kMaxCtas) * QT * pool_capacity(k) * sizeof(uint64_t);
+    return static_cast<size_t>(kMaxCtas) * QT * pp.P * sizeof(uint64_t);
 }
 
 si_status check_common(const void* q, const float* w, const void* kc, int64_t B, int64_t S, int64_t T,
@@ -141,7 +156,8 @@ si_status launch_select_t(const void* q, const float* w, const void* kc, int64_t
     p.T = T;
     p.m = m;
     p.k = dense ? 1 : k;
-    p.P = pool_capacity(p.k);
+    const PoolPlan pp = dense ? PoolPlan{true, 0} : pool_plan(H, D, p.k);
+    p.P = pp.P;
     p.nblk = (S + C::QT - 1) / C::QT;
     p.units = B * p.nblk;
     p.out_idx = out_idx;
@@ -149,9 +165,15 @@ si_status launch_select_t(const void* q, const float* w, const void* kc, int64_t
     p.dense = dense;
     p.err = static_cast<uint32_t*>(ws);
     p.timeout_ns = g_timeout_ns.load();
-    const bool smem_pool = dense || pool_fits_smem(H, D, p.k);
+    const bool smem_pool = pp.smem;
     p.gpool = smem_pool ? nullptr
                         : reinterpret_cast<uint64_t*>(static_cast<uint8_t*>(ws) + kHeaderBytes);
+#ifdef SI_TRACE
+    // Tracing builds: per-warp cycle counters after the pools; the caller adds
+    // kMaxCtas * kTraceWarps * kTraceSlots * 8 bytes to the workspace.
+    p.trace = reinterpret_cast<unsigned long long*>(static_cast<uint8_t*>(ws) + kHeaderBytes +
+                                                    (smem_pool ? 0 : global_pool_bytes(H, D, p.k)));
+#endif
 
     CUtensorMap tq, tkc, tw;
     const uint64_t bf = 2;
@@ -165,10 +187,10 @@ si_status launch_select_t(const void* q, const float* w, const void* kc, int64_t
                    H, C::QT, CU_TENSOR_MAP_SWIZZLE_NONE))
         return SI_ERR_CUDA;
 
-    uint32_t smem = C::smem_bytes(smem_pool, p.P);
+    uint32_t smem = C::dyn_bytes(smem_pool, p.P);
     if (smem < kMinDynSmem) smem = kMinDynSmem;
-    if (smem > kMaxDynSmem) return SI_ERR_UNSUPPORTED;
-    auto kern = si::select_kernel<H, D>;
+    if (smem + C::STATIC_BYTES > kMaxDynSmem) return SI_ERR_UNSUPPORTED;
+    auto kern = smem_pool ? si::select_kernel<H, D, true> : si::select_kernel<H, D, false>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
         cudaSuccess)
         return SI_ERR_CUDA;

@@ -53,8 +53,8 @@ def test_workspace_bytes_host_arithmetic(lib):
     # pools fit in shared memory: header only
     assert si.workspace_bytes(1, 262144, 65536, 64, 128, 4, 512) == 256
     assert si.workspace_bytes(1, 2048, 512, 8, 64, 4, 64) == 256
-    # k = 2048 at H_I=64: 148 CTAs x 4 queries x 4096-entry pools x 8 bytes
-    assert si.workspace_bytes(4, 131072, 32768, 64, 128, 4, 2048) == 256 + 148 * 4 * 4096 * 8
+    # k = 2048 at H_I=64: 148 CTAs x 4 queries x 8192-entry (4k) pools x 8 bytes
+    assert si.workspace_bytes(4, 131072, 32768, 64, 128, 4, 2048) == 256 + 148 * 4 * 8192 * 8
     # independent of S and T (never O(S*T))
     assert si.workspace_bytes(1, 1 << 20, 1 << 18, 64, 128, 4, 2048) == si.workspace_bytes(1, 64, 16, 64, 128, 4, 2048)
     for bad in [(1, 10, 4, 12, 128, 4, 8), (1, 10, 4, 64, 96, 4, 8), (1, 10, 4, 64, 128, 4, 0),
