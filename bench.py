@@ -59,13 +59,16 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+SELECT_SOURCES = ("si_select.cuh", "si_ptx.cuh", "si_keys.cuh")
+
+
 def csrc_hash() -> str:
+    """Hash of the sources the select kernel is built from."""
     d = os.path.join(ROOT, "streaming_top_indexer_b200", "csrc")
     h = hashlib.sha256()
-    for name in sorted(os.listdir(d)):
-        if name.endswith((".cu", ".cuh")):
-            with open(os.path.join(d, name), "rb") as f:
-                h.update(name.encode() + f.read())
+    for name in SELECT_SOURCES:
+        with open(os.path.join(d, name), "rb") as f:
+            h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
 
 

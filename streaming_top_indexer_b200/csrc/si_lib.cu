@@ -191,6 +191,9 @@ si_status launch_select_t(const void* q, const float* w, const void* kc, int64_t
     if (smem < kMinDynSmem) smem = kMinDynSmem;
     if (smem + C::STATIC_BYTES > kMaxDynSmem) return SI_ERR_UNSUPPORTED;
     auto kern = smem_pool ? si::select_kernel<H, D, true> : si::select_kernel<H, D, false>;
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return SI_ERR_CUDA;
+    if (fa.sharedSizeBytes > C::STATIC_BYTES) return SI_ERR_UNSUPPORTED;  // build drifted past the bound
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
         cudaSuccess)
         return SI_ERR_CUDA;

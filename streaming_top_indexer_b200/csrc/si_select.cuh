@@ -111,7 +111,9 @@ struct SelCfg {
     static constexpr uint32_t OFF_POOL = OFF_W + 2 * W_BYTES;
     static constexpr uint32_t ALIGN_SLACK = 1024;
     // static shared memory: barriers, counters, thresholds, histograms
-    static constexpr uint32_t STATIC_BYTES = 10240;  // >= actual static use
+    // Upper bound of the kernel's static shared memory (the host checks the
+    // real figure at launch; pools in shared memory are sized with this).
+    static constexpr uint32_t STATIC_BYTES = 6144;
     static constexpr uint32_t dyn_bytes(bool pool_in_smem, int P) {
         return OFF_POOL + (pool_in_smem ? static_cast<uint32_t>(QT) * P * 8u : 0u) + ALIGN_SLACK;
     }
@@ -243,39 +245,134 @@ struct PoolRegions {
     __device__ __forceinline__ int total() const { return len[0] + len[1] + len[2] + len[3] + len[4]; }
 };
 
+// Per-half scratch of a pool cut, in shared memory.
+struct CutScratch {
+    unsigned long long srt[32];   // 32 samples sorted descending; 0 (below any key) past the last
+    unsigned long long cand[64];  // keys between two adjacent samples (exact cut)
+    unsigned long long xch[8];    // cross-warp exchange
+    uint32_t hist[256];           // radix fallback histogram
+    uint32_t rcnt[2][4];          // per-warp counts, double-buffered by call parity
+    uint32_t ncand;
+};
+
 // Calls f(x) for every key of the regions that thread `tid` of the half owns
-// (virtual positions tid, tid+128, ...), four loads in flight at a time.
+// (virtual positions tid, tid+128, ...).
 template <typename F>
 __device__ __forceinline__ void half_for_each(const uint64_t* pool, const PoolRegions& rg, int tid, F f) {
-#pragma unroll 1
+#pragma unroll
     for (int r = 0; r < 5; ++r) {
         const uint64_t* base = pool + rg.start[r];
         const int len = rg.len[r];
-        int i = tid;
-        for (; i + 384 < len; i += 512) {
-            const uint64_t x0 = base[i], x1 = base[i + 128], x2 = base[i + 256], x3 = base[i + 384];
-            f(x0);
-            f(x1);
-            f(x2);
-            f(x3);
-        }
-        for (; i < len; i += 128) f(base[i]);
+#pragma unroll 2
+        for (int i = tid; i < len; i += 128) f(base[i]);
     }
 }
 
-// Lower bound L of the k best of the n (> k, distinct) keys in the regions,
-// computed by the 128 threads of one epilogue half (tid 0..127, named
-// barrier bar_id): at least k and at most k + slack keys are >= L (exactly k
-// when slack == 0).  Radix select from the most significant bit in which the
-// keys differ, 8 bits per pass; each warp fills its own 256-bin histogram
-// (hist[4][256]) and every warp scans the sum itself, so all threads reach
-// the same decision without a broadcast.  It stops at the first pass whose
-// bucket holding the k-th key leaves at most `slack` extra keys above L.
-__device__ __forceinline__ uint64_t half_select_bound(const uint64_t* pool, const PoolRegions& rg, int k,
-                                                      uint32_t slack, uint32_t (*hist)[256],
-                                                      unsigned long long* xch, int tid, uint32_t bar_id) {
+// Address of virtual position v of the address-ordered regions (v < total).
+__device__ __forceinline__ int region_addr(const PoolRegions& rg, int v) {
+    int a = -1;
+#pragma unroll
+    for (int r = 0; r < 5; ++r) {
+        if (a < 0 && v < rg.len[r]) a = rg.start[r] + v;
+        v -= rg.len[r];
+    }
+    return a;
+}
+
+// Sum over the 128 threads of the half, with one barrier; `phase` selects the
+// exchange buffer and must advance identically in every thread.
+__device__ __forceinline__ uint32_t half_sum(uint32_t c, CutScratch& cs, int tid, uint32_t bar_id, uint32_t& phase) {
     const int lane = tid & 31, wq = tid >> 5;
-    uint32_t* my_hist = hist[wq];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+    uint32_t* rc = cs.rcnt[phase & 1u];
+    ++phase;
+    if (lane == 0) rc[wq] = c;
+    bar_sync(bar_id, 128);
+    return rc[0] + rc[1] + rc[2] + rc[3];
+}
+
+// Key sources of a cut: the pool read from memory on every pass, or the
+// pool's keys held in registers (kRegKeys per thread, pools up to 2048).
+struct StreamKeys {
+    const uint64_t* pool;
+    PoolRegions rg;
+    template <typename F>
+    __device__ __forceinline__ void for_each(int tid, F f) const {
+        half_for_each(pool, rg, tid, f);
+    }
+};
+
+constexpr int kRegKeys = 16;
+
+struct RegKeys {
+    uint64_t x[kRegKeys];
+    int n;
+    __device__ __forceinline__ void load(const uint64_t* pool, const PoolRegions& rg, int tid) {
+        n = rg.total();
+#pragma unroll
+        for (int j = 0; j < kRegKeys; ++j) {
+            const int v = j * 128 + tid;
+            x[j] = v < n ? pool[region_addr(rg, v)] : 0ull;
+        }
+    }
+    template <typename F>
+    __device__ __forceinline__ void for_each(int tid, F f) const {
+#pragma unroll
+        for (int j = 0; j < kRegKeys; ++j)
+            if (j * 128 + tid < n) f(x[j]);
+    }
+};
+
+// Number of keys >= L (every thread of the half gets it).
+template <typename Keys>
+__device__ __forceinline__ uint32_t half_count_ge(const Keys& keys, uint64_t L, CutScratch& cs, int tid,
+                                                  uint32_t bar_id, uint32_t& phase) {
+    uint32_t c = 0;
+    keys.for_each(tid, [&](uint64_t x) { c += x >= L ? 1u : 0u; });
+    return half_sum(c, cs, tid, bar_id, phase);
+}
+
+// Warp-wide bitonic sort, descending, of 32*E keys: element i is v[i/32] of lane i%32.
+template <int E>
+__device__ __forceinline__ void warp_sort_desc(uint64_t (&v)[E], int lane) {
+#pragma unroll
+    for (int size = 2; size <= 32 * E; size <<= 1) {
+#pragma unroll
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            if (stride >= 32) {
+                const int es = stride >> 5;
+#pragma unroll
+                for (int e = 0; e < E; ++e) {
+                    const int pe = e ^ es;
+                    if (pe > e) {
+                        const bool desc = ((e * 32) & size) == 0;
+                        const uint64_t a = v[e], b = v[pe];
+                        const bool sw = desc ? (a < b) : (a > b);
+                        v[e] = sw ? b : a;
+                        v[pe] = sw ? a : b;
+                    }
+                }
+            } else {
+#pragma unroll
+                for (int e = 0; e < E; ++e) {
+                    const int i = e * 32 + lane;
+                    const uint64_t o = __shfl_xor_sync(0xffffffffu, v[e], stride);
+                    const bool take_max = ((lane & stride) == 0) == ((i & size) == 0);
+                    v[e] = take_max ? (v[e] > o ? v[e] : o) : (v[e] < o ? v[e] : o);
+                }
+            }
+        }
+    }
+}
+
+// Radix select (fallback): lower bound L with k <= #(keys >= L) <= k + slack,
+// by the 128 threads of the half.  8 bits per pass from the most significant
+// bit in which the keys differ, on a shared 256-bin histogram; every warp
+// scans the histogram itself, so all threads reach the same decision.
+__device__ __noinline__ uint64_t half_radix_bound(const uint64_t* pool, const PoolRegions& rg, int k, uint32_t slack,
+                                                  CutScratch& cs, int tid, uint32_t bar_id) {
+    const int lane = tid & 31, wq = tid >> 5;
     uint64_t kmin = ~0ull, kmax = 0ull;
     half_for_each(pool, rg, tid, [&](uint64_t x) {
         kmin = x < kmin ? x : kmin;
@@ -289,16 +386,16 @@ __device__ __forceinline__ uint64_t half_select_bound(const uint64_t* pool, cons
         kmax = b > kmax ? b : kmax;
     }
     if (lane == 0) {
-        xch[wq] = kmin;
-        xch[4 + wq] = kmax;
+        cs.xch[wq] = kmin;
+        cs.xch[4 + wq] = kmax;
     }
-#pragma unroll
-    for (int j = 0; j < 8; ++j) my_hist[lane + 32 * j] = 0;
+    cs.hist[tid] = 0;
+    cs.hist[tid + 128] = 0;
     bar_sync(bar_id, 128);
 #pragma unroll
     for (int w = 0; w < 4; ++w) {
-        kmin = xch[w] < kmin ? xch[w] : kmin;
-        kmax = xch[4 + w] > kmax ? xch[4 + w] : kmax;
+        kmin = cs.xch[w] < kmin ? cs.xch[w] : kmin;
+        kmax = cs.xch[4 + w] > kmax ? cs.xch[4 + w] : kmax;
     }
     const int hb = 63 - __clzll(static_cast<long long>(kmin ^ kmax));
     uint64_t dmask = (hb >= 63) ? 0ull : ~((2ull << hb) - 1ull);  // decided bits
@@ -310,16 +407,14 @@ __device__ __forceinline__ uint64_t half_select_bound(const uint64_t* pool, cons
         const int width = lo - shift;
         const uint64_t dig_mask = (1ull << width) - 1ull;
         half_for_each(pool, rg, tid, [&](uint64_t x) {
-            if ((x & dmask) == prefix) atomicAdd(&my_hist[(x >> shift) & dig_mask], 1u);
+            if ((x & dmask) == prefix) atomicAdd(&cs.hist[(x >> shift) & dig_mask], 1u);
         });
         bar_sync(bar_id, 128);
-        // Scan the 256 bins from the top: lane l owns bins 255-8l .. 248-8l.
         uint32_t c[8];
         uint32_t sum = 0;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-            const int bin = 255 - lane * 8 - j;
-            c[j] = hist[0][bin] + hist[1][bin] + hist[2][bin] + hist[3][bin];
+            c[j] = cs.hist[255 - lane * 8 - j];
             sum += c[j];
         }
         uint32_t incl = sum;
@@ -352,63 +447,219 @@ __device__ __forceinline__ uint64_t half_select_bound(const uint64_t* pool, cons
         prefix |= static_cast<uint64_t>(digit) << shift;
         dmask |= dig_mask << shift;
         lo = shift;
-        // every thread has read the histograms before anyone clears them again
-        bar_sync(bar_id, 128);
+        bar_sync(bar_id, 128);  // every thread has read the histogram
         if (cnt - need <= slack || lo == 0) break;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) my_hist[lane + 32 * j] = 0;
-        __syncwarp();
+        cs.hist[tid] = 0;
+        cs.hist[tid + 128] = 0;
+        bar_sync(bar_id, 128);
     }
     return prefix;  // decided bits of the bucket, zeros below: its lowest key
 }
 
-// Walks the region entries >= L in address order, 512 at a time (four per
-// thread), and hands each kept entry with its output position to `emit`; the
-// 128 threads of the half cooperate (per-warp counts exchanged through
-// rcnt[2][4], double-buffered by round parity).  Returns the number kept.
+// Lower bound L of the best keys in the regions, by the 128 threads of one
+// epilogue half: k <= #(keys >= L) <= max_keep (max_keep == k: exactly the k
+// best).  Needs n > k.
+//  1. Warp 0 draws 32 evenly spaced keys and sorts them in registers.
+//  2. Counting passes (one barrier each) test samples near the rank that
+//     predicts the target count, stepping one sample at a time, until a
+//     sample qualifies or two adjacent samples bracket the k-th key.
+//  3. Exact cut: the keys between the bracketing samples (about n/32) are
+//     gathered and one warp sorts them to pick the k-th.
+//  4. A bracket holding more than 64 keys falls back to the radix select.
+template <typename Keys>
+__device__ __forceinline__ uint64_t half_select_bound(const Keys& keys, const uint64_t* pool, const PoolRegions& rg,
+                                                      int k, uint32_t max_keep, CutScratch& cs, int tid,
+                                                      uint32_t bar_id, uint32_t& phase) {
+    const int lane = tid & 31;
+    const int n = rg.total();
+    const int ns = n < 32 ? n : 32;
+    if (tid < 32) {
+        uint64_t v[1];
+        v[0] = lane < ns ? pool[region_addr(rg, n >= 32 ? (lane * n) >> 5 : lane)] : 0ull;
+        warp_sort_desc<1>(v, lane);
+        cs.srt[lane] = v[0];
+    }
+    if (tid == 0) cs.ncand = 0;
+    bar_sync(bar_id, 128);
+    // c(r) = #(keys >= srt[r]) grows with r; c(-1) = 0 (no bound), c(ns) = n (bound 0)
+    const uint32_t ku = static_cast<uint32_t>(k);
+    const uint32_t target = max_keep > ku ? (ku + max_keep) / 2u : ku;
+    int r = static_cast<int>((static_cast<long long>(target) * ns + n - 1) / n) - 1;
+    r = r < 0 ? 0 : (r > ns - 1 ? ns - 1 : r);
+    int lo_r = -1, hi_r = ns;
+    uint32_t c_lo = 0, c_hi = static_cast<uint32_t>(n);
+    for (int it = 0; it < 8; ++it) {
+        const uint32_t c = half_count_ge(keys, cs.srt[r], cs, tid, bar_id, phase);
+        if (c >= ku && c <= max_keep) return cs.srt[r];
+        if (c < ku) {
+            lo_r = r;
+            c_lo = c;
+            ++r;
+        } else {
+            hi_r = r;
+            c_hi = c;
+            --r;
+        }
+        if (r <= lo_r || r >= hi_r) break;
+    }
+    const uint32_t m = c_hi - c_lo;  // keys in [lower, upper)
+    if (hi_r - lo_r != 1 || m > 64u) {
+        bar_sync(bar_id, 128);
+        return half_radix_bound(pool, rg, k, max_keep - ku, cs, tid, bar_id);
+    }
+    const uint64_t upper = lo_r >= 0 ? cs.srt[lo_r] : ~0ull;
+    const uint64_t lower = hi_r < ns ? cs.srt[hi_r] : 0ull;
+    keys.for_each(tid, [&](uint64_t x) {
+        if (x >= lower && x < upper) cs.cand[atomicAdd(&cs.ncand, 1u)] = x;
+    });
+    bar_sync(bar_id, 128);
+    if (tid < 32) {
+        uint64_t v[2];
+        v[0] = lane < static_cast<int>(m) ? cs.cand[lane] : 0ull;
+        v[1] = lane + 32 < static_cast<int>(m) ? cs.cand[lane + 32] : 0ull;
+        warp_sort_desc<2>(v, lane);
+        const int want = static_cast<int>(ku - c_lo) - 1;  // 0-based rank inside the bracket
+        if (lane == want) cs.xch[0] = v[0];
+        if (lane + 32 == want) cs.xch[0] = v[1];
+    }
+    bar_sync(bar_id, 128);
+    return cs.xch[0];
+}
+
+// Hands every region entry >= L, with a distinct output position in
+// [0, kept), to `emit`, by the 128 threads of the half; returns kept.
+// Positions are assigned per warp in blocks (entry order is not kept).  Each
+// chunk of 2048 entries is loaded into registers before one barrier and
+// written after it, so packing the pool into its own front is safe in place:
+// a chunk's writes never reach past its own entries.
 template <typename Emit>
 __device__ __forceinline__ uint32_t half_walk_kept(const uint64_t* pool, const PoolRegions& rg, uint64_t L,
-                                                   uint32_t* rcnt, int tid, uint32_t bar_id, Emit emit) {
+                                                   CutScratch& cs, int tid, uint32_t bar_id, uint32_t& phase,
+                                                   Emit emit) {
+    constexpr int EP = 16;  // entries per thread per chunk
     const int lane = tid & 31, wq = tid >> 5;
-    const uint32_t lt = lanemask_lt();
-    uint32_t out = 0, round = 0;
-#pragma unroll 1
-    for (int r = 0; r < 5; ++r) {
-        const uint64_t* base = pool + rg.start[r];
-        const int len = rg.len[r];
-        for (int b0 = 0; b0 < len; b0 += 512) {
-            // this warp's 128 consecutive entries: four groups of 32
-            uint64_t x[4];
-            uint32_t bal[4];
-            uint32_t mine = 0;
+    const int n = rg.total();
+    uint32_t out = 0;
+    for (int c0 = 0; c0 < n; c0 += 128 * EP) {
+        uint64_t x[EP];
+        uint32_t keep = 0, mine = 0;
 #pragma unroll
-            for (int g = 0; g < 4; ++g) {
-                const int i = b0 + wq * 128 + g * 32 + lane;
-                const bool in = i < len;
-                x[g] = in ? base[i] : 0ull;
-                bal[g] = __ballot_sync(0xffffffffu, in && x[g] >= L);
-                mine += static_cast<uint32_t>(__popc(bal[g]));
-            }
-            uint32_t* rc = rcnt + (round & 1u) * 4u;
-            if (lane == 0) rc[wq] = mine;
-            bar_sync(bar_id, 128);
-            uint32_t pos = out, total = 0;
-#pragma unroll
-            for (int w = 0; w < 4; ++w) {
-                const uint32_t cw = rc[w];
-                pos += (w < wq) ? cw : 0u;
-                total += cw;
-            }
-#pragma unroll
-            for (int g = 0; g < 4; ++g) {
-                if ((bal[g] >> lane) & 1u) emit(x[g], pos + static_cast<uint32_t>(__popc(bal[g] & lt)));
-                pos += static_cast<uint32_t>(__popc(bal[g]));
-            }
-            out += total;
-            ++round;
+        for (int j = 0; j < EP; ++j) {
+            const int v = c0 + j * 128 + tid;
+            x[j] = v < n ? pool[region_addr(rg, v)] : 0ull;
+            const bool kp = v < n && x[j] >= L;
+            keep |= (kp ? 1u : 0u) << j;
+            mine += kp ? 1u : 0u;
         }
+        // exclusive prefix of `mine` over the warp, and per-warp totals
+        uint32_t incl = mine;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += t;
+        }
+        const uint32_t wtot = __shfl_sync(0xffffffffu, incl, 31);
+        uint32_t* rc = cs.rcnt[phase & 1u];
+        ++phase;
+        if (lane == 0) rc[wq] = wtot;
+        bar_sync(bar_id, 128);
+        uint32_t pos = out + incl - mine, total = 0;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+            const uint32_t cw = rc[w];
+            pos += (w < wq) ? cw : 0u;
+            total += cw;
+        }
+#pragma unroll
+        for (int j = 0; j < EP; ++j)
+            if ((keep >> j) & 1u) emit(x[j], pos++);
+        out += total;
     }
     return out;
+}
+
+// half_walk_kept for keys held in registers: one barrier, then each thread
+// emits its kept keys (safe in place: every key was read before).
+template <typename Emit>
+__device__ __forceinline__ uint32_t half_walk_reg(const RegKeys& rk, uint64_t L, CutScratch& cs, int tid,
+                                                  uint32_t bar_id, uint32_t& phase, Emit emit) {
+    const int lane = tid & 31, wq = tid >> 5;
+    uint32_t keep = 0, mine = 0;
+#pragma unroll
+    for (int j = 0; j < kRegKeys; ++j) {
+        const bool kp = j * 128 + tid < rk.n && rk.x[j] >= L;
+        keep |= (kp ? 1u : 0u) << j;
+        mine += kp ? 1u : 0u;
+    }
+    uint32_t incl = mine;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+    }
+    const uint32_t wtot = __shfl_sync(0xffffffffu, incl, 31);
+    uint32_t* rc = cs.rcnt[phase & 1u];
+    ++phase;
+    if (lane == 0) rc[wq] = wtot;
+    bar_sync(bar_id, 128);
+    uint32_t pos = incl - mine, total = 0;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+        const uint32_t cw = rc[w];
+        pos += (w < wq) ? cw : 0u;
+        total += cw;
+    }
+#pragma unroll
+    for (int j = 0; j < kRegKeys; ++j)
+        if ((keep >> j) & 1u) emit(rk.x[j], pos++);
+    return total;
+}
+
+// Cuts one query's pool to its best keys -- between k and max_keep of them,
+// or all when there are at most k -- packed at the front of the pool, by the
+// 128 threads of the half.  Returns the new lower bound; `kept` gets the count.
+__device__ __noinline__ uint64_t cut_pool(uint64_t* pq, PoolRegions rg, int k, uint32_t max_keep, uint64_t lb,
+                                          CutScratch& cs, int tid, uint32_t bar_id, uint32_t& phase,
+                                          uint32_t& kept) {
+    uint64_t L = lb;
+    if (rg.total() <= 128 * kRegKeys) {
+        RegKeys rk;
+        rk.load(pq, rg, tid);
+        if (rk.n > k) L = half_select_bound(rk, pq, rg, k, max_keep, cs, tid, bar_id, phase);
+        kept = half_walk_reg(rk, L, cs, tid, bar_id, phase, [&](uint64_t x, uint32_t pos) { pq[pos] = x; });
+    } else {
+        const StreamKeys sk{pq, rg};
+        if (rg.total() > k) L = half_select_bound(sk, pq, rg, k, max_keep, cs, tid, bar_id, phase);
+        kept = half_walk_kept(pq, rg, L, cs, tid, bar_id, phase, [&](uint64_t x, uint32_t pos) { pq[pos] = x; });
+    }
+    return L;
+}
+
+// Writes the k best keys of one query's pool (or all, when fewer), unordered,
+// to its output row, then pads the row with (-1, -inf); by the half.
+__device__ __noinline__ void emit_best(const uint64_t* pq, PoolRegions rg, int k, CutScratch& cs, int tid,
+                                       uint32_t bar_id, uint32_t& phase, int32_t* out_idx, float* out_score) {
+    auto emit = [&](uint64_t x, uint32_t pos) {
+        out_idx[pos] = key_index(x);
+        out_score[pos] = key_score(x);
+    };
+    uint32_t out;
+    if (rg.total() <= 128 * kRegKeys) {
+        RegKeys rk;
+        rk.load(pq, rg, tid);
+        const uint64_t L = rk.n > k ? half_select_bound(rk, pq, rg, k, static_cast<uint32_t>(k), cs, tid, bar_id, phase)
+                                    : 0ull;
+        out = half_walk_reg(rk, L, cs, tid, bar_id, phase, emit);
+    } else {
+        const StreamKeys sk{pq, rg};
+        const uint64_t L =
+            rg.total() > k ? half_select_bound(sk, pq, rg, k, static_cast<uint32_t>(k), cs, tid, bar_id, phase) : 0ull;
+        out = half_walk_kept(pq, rg, L, cs, tid, bar_id, phase, emit);
+    }
+    for (int i = static_cast<int>(out) + tid; i < k; i += 128) {
+        out_idx[i] = -1;
+        out_score[i] = -__int_as_float(0x7f800000);
+    }
 }
 
 // Regions of query slot `qi` from the published survivor count and the four
@@ -438,9 +689,7 @@ __global__ void __launch_bounds__(SelCfg<H, D>::THREADS, 1)
     // Pool bookkeeping published at cuts, [half][query of the half]: append
     // counts of the four warps, survivors of the cut and the lower bound.
     __shared__ uint32_t cntw[2][16][4];
-    __shared__ uint32_t hist_s[2][4][256];          // per half and warp: radix histograms
-    __shared__ unsigned long long xch_s[2][8];      // per half: min/max exchange
-    __shared__ uint32_t rcnt_s[2][8];               // per half: warp counts of a walk round
+    __shared__ CutScratch cut_s[2];                 // per half: pool-cut scratch
     SI_TR_DECL;
     SI_TR_T0(t_kernel0);
 
@@ -602,9 +851,8 @@ __global__ void __launch_bounds__(SelCfg<H, D>::THREADS, 1)
         const uint32_t bar_id = 1u + static_cast<uint32_t>(half);
         const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
         const int htid = wih * 32 + lane;  // thread index within the half
-        uint32_t(*hist)[256] = hist_s[half];
-        unsigned long long* xch = xch_s[half];
-        uint32_t* rcnt = rcnt_s[half];
+        CutScratch& cs = cut_s[half];
+        uint32_t cphase = 0;  // exchange-buffer parity of the half's cut helpers
         const bool dense = p.dense != nullptr;
         const int k = p.k;
         const uint32_t Pu = static_cast<uint32_t>(P);
@@ -671,7 +919,6 @@ __global__ void __launch_bounds__(SelCfg<H, D>::THREADS, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar(kBarAccEmpty + buf));
                 SI_TR_ADD(kTrEpiArrive, tar0, tr_lead);
-                SI_TR_T0(tfl0);
                 const int32_t s = j * C::BM + quarter * 32 + lane;
                 bool need = false;
                 if (ok) {
@@ -697,6 +944,7 @@ __global__ void __launch_bounds__(SelCfg<H, D>::THREADS, 1)
                         }
                     }
                 }
+                SI_TR_T0(tfl0);
                 // One barrier per tile (abort and cut requests are OR-reduced);
                 // two more only when some sub-range is nearly full or a wait failed.
                 const bool bad_here = !ok || *abort_flag;
@@ -723,19 +971,10 @@ __global__ void __launch_bounds__(SelCfg<H, D>::THREADS, 1)
                         const bool cut = c4[0] + 32u > f || c4[1] + 32u > f || c4[2] + 32u > f || c4[3] + 32u > f;
                         if (!cut) continue;  // uniform over the half
                         uint64_t* pq = pool + (half * C::QH + q) * P;
-                        const PoolRegions rg = pool_regions(kp[q], f, c4);
-                        uint64_t L = lb[q];
-                        SI_TR_T0(tsel0);
-                        if (rg.total() > k) L = half_select_bound(pq, rg, k, cut_slack, hist, xch, htid, bar_id);
-                        SI_TR_ADD(0, tsel0, true);
-                        SI_TR_T0(twk0);
-                        const uint32_t kept = half_walk_kept(pq, rg, L, rcnt, htid, bar_id,
-                                                             [&](uint64_t x, uint32_t pos) { pq[pos] = x; });
-                        SI_TR_ADD(1, twk0, true);
-#ifdef SI_TRACE
-                        tr_acc[3] += static_cast<unsigned long long>(rg.total());
-                        tr_acc[4] += kept;
-#endif
+                        uint32_t kept = 0;
+                        const uint64_t L = cut_pool(pq, pool_regions(kp[q], f, c4), k,
+                                                    static_cast<uint32_t>(k) + cut_slack, lb[q], cs, htid, bar_id,
+                                                    cphase, kept);
                         SI_TR_INC(kTrCompactions, true);
                         kp[q] = kept;
                         lb[q] = L;
@@ -761,20 +1000,9 @@ __global__ void __launch_bounds__(SelCfg<H, D>::THREADS, 1)
                     const int qi = half * C::QH + q;
                     const int64_t t = ui.t0 + qi;
                     if (t >= p.S) continue;  // uniform over the half
-                    const uint64_t* pq = pool + qi * P;
-                    const PoolRegions rg = pool_regions(kp[q], fw(q), cntw[half][q]);
-                    const uint64_t L =
-                        rg.total() > k ? half_select_bound(pq, rg, k, 0u, hist, xch, htid, bar_id) : 0ull;
                     const int64_t row = (ui.b * p.S + t) * static_cast<int64_t>(k);
-                    // The k best (or all, when fewer), unordered, then padding.
-                    const uint32_t out = half_walk_kept(pq, rg, L, rcnt, htid, bar_id, [&](uint64_t x, uint32_t pos) {
-                        p.out_idx[row + pos] = key_index(x);
-                        p.out_score[row + pos] = key_score(x);
-                    });
-                    for (int i = static_cast<int>(out) + htid; i < k; i += 128) {
-                        p.out_idx[row + i] = -1;
-                        p.out_score[row + i] = -__int_as_float(0x7f800000);
-                    }
+                    emit_best(pool + qi * P, pool_regions(kp[q], fw(q), cntw[half][q]), k, cs, htid, bar_id, cphase,
+                              p.out_idx + row, p.out_score + row);
                     bar_sync(bar_id, 128);
                 }
             }
