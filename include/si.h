@@ -111,6 +111,33 @@ SI_API si_status si_check_device_status(const void* workspace, si_stream_t strea
 SI_API si_status si_selftest_timeout(void* workspace, size_t workspace_bytes, uint64_t limit_ns,
                               si_stream_t stream);
 
+/* si_indexer_topk without a caller-supplied workspace, for callers that
+ * cannot allocate device memory themselves (for instance a plugin inside a
+ * host application that owns all device memory, or a serving loop whose
+ * memory plan is fixed after start-up).  The paper has no counterpart; this
+ * is a packaging variant of the same computation and results.
+ *
+ * Scratch: a fixed 1 MiB array in device memory, one per device, that every
+ * device which loads this library keeps until the process exits.  The call
+ * allocates nothing (no cudaMalloc, cudaFree or allocating library routine).
+ * The first call on a device looks up that array's device address (with the
+ * device current) and remembers it; that first call on a device should come
+ * before any stream capture.  All calls on a device share the
+ * array, which keeps the last call's contents; the call clears what must
+ * start at zero.  Calls whose work overlaps on the GPU (different streams,
+ * no ordering between them) race on the shared array: order them.
+ *
+ * Limit: configurations whose si_workspace_bytes() exceeds 1 MiB -- those
+ * whose candidate pools do not fit in shared memory, e.g. k > 512 at
+ * H_I=64, d_I=128 -- return SI_ERR_WORKSPACE_TOO_SMALL before anything is
+ * enqueued.  Everything else is as si_indexer_topk.  out_status, if not NULL,
+ * is a device word that receives the device status of the call (0, or
+ * SI_ERR_TIMEOUT) once the stream reaches the end of the call. */
+SI_API si_status si_indexer_topk_noalloc(const void* q, const float* w, const void* kc,
+                                         int64_t B, int64_t S, int64_t T, int H_I, int d_I, int m, int k,
+                                         int32_t* out_idx, float* out_score, uint32_t* out_status,
+                                         si_stream_t stream);
+
 /* Device-side wait limit, in nanoseconds, used by later calls (default 2 s). */
 SI_API void si_set_timeout_ns(uint64_t ns);
 

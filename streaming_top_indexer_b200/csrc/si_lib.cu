@@ -339,3 +339,71 @@ const char* si_status_string(si_status s) {
 const char* si_version(void) { return "streaming_top_indexer_b200 0.1.0 (sm_100a)"; }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Variant that needs no caller-allocated workspace.
+//
+// Some callers cannot hand the library a device buffer: a plugin running
+// inside a host application that owns every byte of device memory and gives
+// plugins no allocator, or a serving loop whose memory plan is frozen after
+// start-up.  For them the scratch that si_indexer_topk keeps in the caller's
+// workspace (the device error word, plus candidate pools when they do not fit
+// in shared memory) lives instead in the fixed array below, one per device.
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t{1} << 20;  // 1 MiB on every device that loads the library
+
+// Device-side storage.  In host code this name only stands for the symbol;
+// its device address comes from cudaGetSymbolAddress below.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[64] = {};
+
+// Device address of g_noalloc_scratch on the current device, looked up once
+// per device (with that device current) and remembered.
+si_status noalloc_scratch(void** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return SI_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (g_noalloc_addr[dev] == nullptr) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return SI_ERR_CUDA;
+        g_noalloc_addr[dev] = p;
+    }
+    *out = g_noalloc_addr[dev];
+    return SI_OK;
+}
+
+}  // namespace
+
+extern "C" si_status si_indexer_topk_noalloc(const void* q, const float* w, const void* kc, int64_t B, int64_t S,
+                                             int64_t T, int H_I, int d_I, int m, int k, int32_t* out_idx,
+                                             float* out_score, uint32_t* out_status, si_stream_t stream) {
+    si_status st = check_common(q, w, kc, B, S, T, H_I, d_I, m);
+    if (st != SI_OK) return st;
+    if (k < 1 || k > 2048) return SI_ERR_UNSUPPORTED;
+    if (!out_idx || !out_score) return SI_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(out_idx) & 3u) || (reinterpret_cast<uintptr_t>(out_score) & 3u) ||
+        (reinterpret_cast<uintptr_t>(out_status) & 3u))
+        return SI_ERR_MISALIGNED;
+    const size_t need = si_workspace_bytes(B, S, T, H_I, d_I, m, k);
+    if (need == 0) return SI_ERR_UNSUPPORTED;
+    if (need > kNoAllocScratchBytes) return SI_ERR_WORKSPACE_TOO_SMALL;  // beyond the built-in scratch
+    void* ws = nullptr;
+    st = noalloc_scratch(&ws);
+    if (st != SI_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    // The array keeps the previous call's contents: clear the error word.
+    if (cudaMemsetAsync(ws, 0, kHeaderBytes, s) != cudaSuccess) return SI_ERR_CUDA;
+    if (T == 0) {
+        st = launch_pad(out_idx, out_score, B * S * k, s);
+    } else {
+        st = launch_select(q, w, kc, B, S, T, H_I, d_I, m, k, out_idx, out_score, nullptr, ws, s);
+        if (st == SI_OK) st = si_sort_topk(out_idx, out_score, B * S, k, stream);
+    }
+    if (st != SI_OK) return st;
+    if (out_status && cudaMemcpyAsync(out_status, ws, sizeof(uint32_t), cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+        return SI_ERR_CUDA;
+    return SI_OK;
+}
