@@ -140,6 +140,16 @@ def test_timeout_selftest_reports_and_context_survives():
     assert idx.shape == (1, 256, 8)
 
 
+def test_workspace_pools_with_streamed_cuts():
+    """k=1024 at H_I=64 puts the candidate pools in the workspace (4k entries
+    per query), and rows long enough that the pools are cut while more than
+    2048 entries are held: the streamed (not register-held) cut path."""
+    wl = synth.Workload("ws_pools", 1, 98304, 4, 64, 128, 1024)
+    q, w, kc = synth.generate(wl, seed=21, device=DEV)
+    b_rows, t_rows = gh.sampled_rows(wl.B, wl.S, wl.m, wl.k, n=256)
+    gh.check_against_oracle(q, w, kc, wl.m, wl.k, b_rows, t_rows, where="ws pools")
+
+
 @pytest.mark.parametrize("name", ["v4flash", "long"])
 def test_full_size_sampled_rows(name):
     """Full-size workloads in the benchmark's launch configuration: 512
