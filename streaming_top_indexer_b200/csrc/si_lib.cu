@@ -8,6 +8,8 @@
 
 #include <atomic>
 #include <cstdint>
+#include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -18,6 +20,13 @@
 #include "si_sort.cuh"
 
 namespace {
+
+// With SI_DEBUG set in the environment, CUDA failures are also printed to stderr.
+si_status cuda_fail(const char* where, cudaError_t e) {
+    static const bool verbose = std::getenv("SI_DEBUG") != nullptr;
+    if (verbose) std::fprintf(stderr, "streaming_top_indexer: %s: %s\n", where, cudaGetErrorString(e));
+    return SI_ERR_CUDA;
+}
 
 constexpr int kMaxCtas = 148;                 // persistent CTAs (one per B200 SM)
 constexpr size_t kHeaderBytes = 256;          // error word + reserved
@@ -194,13 +203,13 @@ si_status launch_select_t(const void* q, const float* w, const void* kc, int64_t
     cudaFuncAttributes fa;
     if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return SI_ERR_CUDA;
     if (fa.sharedSizeBytes > C::STATIC_BYTES) return SI_ERR_UNSUPPORTED;  // build drifted past the bound
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
-        cudaSuccess)
-        return SI_ERR_CUDA;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return cuda_fail("select kernel shared-memory attribute", e);
     int64_t grid = sms < kMaxCtas ? sms : kMaxCtas;
     if (grid > p.units) grid = p.units;
     kern<<<static_cast<unsigned>(grid), C::THREADS, smem, stream>>>(tq, tkc, tw, p);
-    return cudaGetLastError() == cudaSuccess ? SI_OK : SI_ERR_CUDA;
+    e = cudaGetLastError();
+    return e == cudaSuccess ? SI_OK : cuda_fail("select kernel launch", e);
 }
 
 si_status launch_select(const void* q, const float* w, const void* kc, int64_t B, int64_t S, int64_t T, int H, int D,

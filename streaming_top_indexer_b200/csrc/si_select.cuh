@@ -92,7 +92,9 @@ struct SelCfg {
     static_assert(D == 64 || D == 128, "d_I");
     static constexpr int N = 256;               // MMA N: queries x heads per unit
     static constexpr int QT = N / H;            // queries per unit
-    static constexpr int QH = QT / 2;           // queries per epilogue half
+    static constexpr int NGROUPS = 2;           // epilogue groups of four warps
+    static constexpr int QH = QT / NGROUPS;     // queries per epilogue group
+    static constexpr int CG = N / NGROUPS;      // TMEM columns per epilogue group
     static constexpr int BM = 128;              // keys per tile (MMA M)
     static constexpr int KCH = D / 64;          // 128-byte K chunks
     static constexpr int STAGES = (D == 64) ? 4 : 3;
@@ -101,8 +103,15 @@ struct SelCfg {
     static constexpr uint32_t Q_BYTES = KCH * Q_CHUNK;
     static constexpr uint32_t KC_BYTES = KCH * KC_CHUNK;
     static constexpr uint32_t W_BYTES = QT * H * 4u;
-    static constexpr int EPI_WARPS = 8;
-    static constexpr int THREADS = 64 + 32 * EPI_WARPS;
+    static constexpr int EPI_WARPS = 4 * NGROUPS;
+    static constexpr int EPI_WARP0 = 4;         // warps 0-3: TMA producer, MMA issuer, two idle
+    static constexpr int THREADS = 32 * EPI_WARP0 + 32 * EPI_WARPS;
+    // Registers: launched at 168 per thread; the control warpgroup then gives
+    // registers up so that each epilogue thread can hold its 128 head weights.
+    static constexpr uint32_t REGS_LAUNCH = 168, REGS_CTRL = 56, REGS_EPI = 224;
+    static_assert(NGROUPS == 2, "register split assumes two epilogue warpgroups");
+    static_assert(REGS_CTRL * 128 + REGS_EPI * 32 * EPI_WARPS == REGS_LAUNCH * THREADS,
+                  "the register split must add up to the launch allocation");
     static constexpr uint32_t TMEM_COLS = 512;  // two 256-column accumulators
     // dynamic shared memory map, relative to a 1024-byte aligned base
     static constexpr uint32_t OFF_Q = 0;
@@ -180,18 +189,41 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
 // Column j of the half is head (j % H) of query (j / H); consecutive heads
 // are paired into one packed f32x2 FMA, pair p of a query goes to partial
 // sum p % NP.
-template <int H, int QH, int NP>
-__device__ __forceinline__ void accumulate_chunk(const uint32_t (&r)[32], int c, const float* wq,
+// How the ReLU of a head pair is computed.  max(x, 0) runs on the ALU pipe,
+// which has half the issue rate of the FMA pipe and also carries the
+// integer work; x + |x| = 2*relu(x) is one FADD on the FMA pipe (the abs is
+// an operand modifier).  Pairs computed the second way accumulate twice the
+// value into their own partial sums, which are halved at the end: scaling by
+// 2 is exact in binary floating point, so the scores are bit-identical either
+// way.  Mode 1 alternates the two ways by head pair (balancing the pipes),
+// mode 2 uses the FADD form for every pair.
+template <int NP>
+struct ReluPlan {
+    static constexpr int MODE = NP >= 2 ? 1 : 2;
+    // partial sum a holds doubled terms
+    static constexpr bool doubled(int a) { return MODE == 2 || (MODE == 1 && (a & 1)); }
+};
+
+__device__ __forceinline__ float relu_max(float x) { return fmaxf(x, 0.0f); }
+__device__ __forceinline__ float relu_twice(float x) { return x + fabsf(x); }
+
+template <int H, int QH, int NP, int CG>
+__device__ __forceinline__ void accumulate_chunk(const uint32_t (&r)[32], int c, const float (&wr)[CG],
                                                  float2 (&acc)[QH][NP]) {
+    using RP = ReluPlan<NP>;
 #pragma unroll
     for (int i = 0; i < 32; i += 4) {
         const int col = c * 32 + i;
         const int q = col / H;
         const int h = col % H;
-        const float4 w4 = *reinterpret_cast<const float4*>(wq + q * H + h);
-        const float2 x01 = make_float2(fmaxf(__uint_as_float(r[i]), 0.0f), fmaxf(__uint_as_float(r[i + 1]), 0.0f));
-        const float2 x23 = make_float2(fmaxf(__uint_as_float(r[i + 2]), 0.0f), fmaxf(__uint_as_float(r[i + 3]), 0.0f));
+        const float4 w4 = make_float4(wr[col], wr[col + 1], wr[col + 2], wr[col + 3]);
         const int p0 = (h / 2) % NP, p1 = (h / 2 + 1) % NP;
+        const float a0 = __uint_as_float(r[i]), a1 = __uint_as_float(r[i + 1]);
+        const float a2 = __uint_as_float(r[i + 2]), a3 = __uint_as_float(r[i + 3]);
+        const float2 x01 = RP::doubled(p0) ? make_float2(relu_twice(a0), relu_twice(a1))
+                                           : make_float2(relu_max(a0), relu_max(a1));
+        const float2 x23 = RP::doubled(p1) ? make_float2(relu_twice(a2), relu_twice(a3))
+                                           : make_float2(relu_max(a2), relu_max(a3));
         acc[q][p0] = __ffma2_rn(make_float2(w4.x, w4.y), x01, acc[q][p0]);
         acc[q][p1] = __ffma2_rn(make_float2(w4.z, w4.w), x23, acc[q][p1]);
     }
@@ -203,8 +235,8 @@ __device__ __forceinline__ void accumulate_chunk(const uint32_t (&r)[32], int c,
 // whatever the key's position in the tile.  `taddr` points at the half's
 // first column in this warp's lane quarter; `wq` at the half's w [QH][H].
 // TMEM loads are software-pipelined two chunks deep.
-template <int H, int QH, int NP>
-__device__ __forceinline__ void half_scores(uint32_t taddr, const float* wq, float (&sc)[QH]) {
+template <int H, int QH, int NP, int NCH>
+__device__ __forceinline__ void half_scores(uint32_t taddr, const float (&wr)[32 * NCH], float (&sc)[QH]) {
     float2 acc[QH][NP];
 #pragma unroll
     for (int q = 0; q < QH; ++q)
@@ -213,21 +245,22 @@ __device__ __forceinline__ void half_scores(uint32_t taddr, const float* wq, flo
     uint32_t ra[32], rb[32];
     tmem_ld32(taddr, ra);
     tmem_wait_ld(ra);
-    tmem_ld32(taddr + 32, rb);
-    accumulate_chunk<H, QH, NP>(ra, 0, wq, acc);
-    tmem_wait_ld(rb);
-    tmem_ld32(taddr + 64, ra);
-    accumulate_chunk<H, QH, NP>(rb, 1, wq, acc);
-    tmem_wait_ld(ra);
-    tmem_ld32(taddr + 96, rb);
-    accumulate_chunk<H, QH, NP>(ra, 2, wq, acc);
-    tmem_wait_ld(rb);
-    accumulate_chunk<H, QH, NP>(rb, 3, wq, acc);
+#pragma unroll
+    for (int c = 0; c < NCH; ++c) {
+        uint32_t(&cur)[32] = (c & 1) ? rb : ra;
+        uint32_t(&nxt)[32] = (c & 1) ? ra : rb;
+        if (c + 1 < NCH) tmem_ld32(taddr + (c + 1) * 32, nxt);
+        accumulate_chunk<H, QH, NP, 32 * NCH>(cur, c, wr, acc);
+        if (c + 1 < NCH) tmem_wait_ld(nxt);
+    }
 #pragma unroll
     for (int q = 0; q < QH; ++q) {
         float part[NP];
 #pragma unroll
-        for (int a = 0; a < NP; ++a) part[a] = acc[q][a].x + acc[q][a].y;
+        for (int a = 0; a < NP; ++a) {
+            part[a] = acc[q][a].x + acc[q][a].y;
+            if (ReluPlan<NP>::doubled(a)) part[a] *= 0.5f;
+        }
 #pragma unroll
         for (int w = 1; w < NP; w *= 2)
 #pragma unroll
@@ -688,8 +721,8 @@ __global__ void __launch_bounds__(SelCfg<H, D>::THREADS, 1)
     __shared__ int abort_flag_s;
     // Pool bookkeeping published at cuts, [half][query of the half]: append
     // counts of the four warps, survivors of the cut and the lower bound.
-    __shared__ uint32_t cntw[2][16][4];
-    __shared__ CutScratch cut_s[2];                 // per half: pool-cut scratch
+    __shared__ uint32_t cntw[C::NGROUPS][C::QH][4];
+    __shared__ CutScratch cut_s[C::NGROUPS];        // per group: pool-cut scratch
     SI_TR_DECL;
     SI_TR_T0(t_kernel0);
 
@@ -738,6 +771,9 @@ __global__ void __launch_bounds__(SelCfg<H, D>::THREADS, 1)
     const int64_t cta = blockIdx.x;
     const int64_t U = p.units;
 
+    if (warp < C::EPI_WARP0) {
+    // The control warpgroup hands registers to the epilogue warpgroups.
+    regs_shrink_to<C::REGS_CTRL>();
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
         if (lane == 0) {
@@ -842,11 +878,13 @@ __global__ void __launch_bounds__(SelCfg<H, D>::THREADS, 1)
             }
         }
         __syncwarp();
+    }
     } else {
         // ------------------------------------------------ epilogue
-        const int e = warp - 2;
+        regs_grow_to<C::REGS_EPI>();
+        const int e = warp - C::EPI_WARP0;
         const int quarter = warp & 3;
-        const int half = e >> 2;
+        const int half = e >> 2;  // epilogue group
         const int wih = e & 3;
         const uint32_t bar_id = 1u + static_cast<uint32_t>(half);
         const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
@@ -899,6 +937,20 @@ __global__ void __launch_bounds__(SelCfg<H, D>::THREADS, 1)
             }
             const float* wq =
                 reinterpret_cast<const float*>(smem + C::OFF_W + wslot * C::W_BYTES) + half * C::QH * H;
+            // The half's head weights stay in registers for the whole unit
+            // (reloaded after a pool cut, whose call does not preserve them).
+            float wr[C::CG];
+            auto load_w = [&]() {
+#pragma unroll
+                for (int i = 0; i < C::CG; i += 4) {
+                    const float4 v = *reinterpret_cast<const float4*>(wq + i);
+                    wr[i] = v.x;
+                    wr[i + 1] = v.y;
+                    wr[i + 2] = v.z;
+                    wr[i + 3] = v.w;
+                }
+            };
+            if (ui.ntiles > 0) load_w();
             for (int j = 0; j < ui.ntiles; ++j) {
                 const uint32_t buf = acc_it & 1u;
                 SI_TR_T0(tf0);
@@ -910,7 +962,7 @@ __global__ void __launch_bounds__(SelCfg<H, D>::THREADS, 1)
                 tc_fence_after();
                 SI_TR_T0(ts0);
                 float sc[C::QH];
-                half_scores<H, C::QH, C::NP>(tmem_base + buf * C::N + half * 128 + lane_off, wq, sc);
+                half_scores<H, C::QH, C::NP, C::CG / 32>(tmem_base + buf * C::N + half * C::CG + lane_off, wr, sc);
 #pragma unroll
                 for (int q = 0; q < C::QH; ++q) SI_TR_DEPF(sc[q]);
                 SI_TR_ADD(kTrEpiScores, ts0, tr_lead);
@@ -981,6 +1033,7 @@ __global__ void __launch_bounds__(SelCfg<H, D>::THREADS, 1)
                         cw[q] = 0u;
                         bar_sync(bar_id, 128);
                     }
+                    load_w();
                     SI_TR_ADD(kTrEpiCompact, tc0, tr_lead);
                 }
             }
