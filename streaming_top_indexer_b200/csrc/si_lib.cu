@@ -49,7 +49,8 @@ uint32_t select_smem(int H, int D, bool pool_in_smem, int P) {
 }
 
 // Where the per-query candidate pools live and how large they are.  A pool
-// holds at least max(2k, k+256) entries; in shared memory it takes all the
+// holds at least max(2k, k+288) entries (room for k + 28 survivors of a cut
+// plus two tiles of appends in each warp's sub-range); in shared memory it takes all the
 // room left (fewer pool cuts), otherwise 4k entries in the workspace.
 struct PoolPlan {
     bool smem;
@@ -58,7 +59,7 @@ struct PoolPlan {
 
 PoolPlan pool_plan(int H, int D, int k) {
     auto r32 = [](int x) { return (x + 31) / 32 * 32; };
-    const int min_p = r32(2 * k > k + 256 ? 2 * k : k + 256);
+    const int min_p = r32(2 * k > k + 288 ? 2 * k : k + 288);
     const uint32_t qt = 256u / static_cast<uint32_t>(H);
     const uint32_t fixed = select_smem(H, D, false, 0);
     if (fixed + qt * static_cast<uint32_t>(min_p) * 8u <= kMaxDynSmem) {
@@ -66,7 +67,7 @@ PoolPlan pool_plan(int H, int D, int k) {
         if (p > 65504) p = 65504;  // pool counts are 16-bit fields
         return {true, p};
     }
-    return {false, r32(4 * k > k + 256 ? 4 * k : k + 256)};
+    return {false, r32(4 * k > k + 288 ? 4 * k : k + 288)};
 }
 
 size_t global_pool_bytes(int H, int D, int k) {

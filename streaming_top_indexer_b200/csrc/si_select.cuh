@@ -74,7 +74,7 @@ __device__ __forceinline__ long long tr_clock() {
 struct SelectParams {
     int64_t B, S, T;
     int m, k;
-    int P;              // pool capacity per query (multiple of 32, >= k + 256)
+    int P;              // pool capacity per query (multiple of 32, >= k + 288)
     int64_t nblk;       // query blocks per batch
     int64_t units;      // B * nblk
     int32_t* out_idx;   // [B,S,k]
@@ -137,6 +137,10 @@ struct SelCfg {
 // Extra entries an intermediate pool cut may keep above k (the cut at the end
 // of a unit is exact).
 constexpr uint32_t kCompactSlack = 256;
+
+// Tiles between two checks of the pools' fill (each check is a named barrier
+// over the epilogue half).
+constexpr uint32_t kCheckTiles = 2;
 
 // Mbarrier slots.
 enum : int {
@@ -895,9 +899,10 @@ __global__ void __launch_bounds__(SelCfg<H, D>::THREADS, 1)
         const int k = p.k;
         const uint32_t Pu = static_cast<uint32_t>(P);
         // An intermediate cut keeps at most k + cut_slack entries, which leaves
-        // every warp's sub-range at least 33 free slots (P >= k + 256).
+        // every warp's sub-range more than kCheckTiles*32 free slots (P >= k + 288).
+        const uint32_t room = 4u * (32u * kCheckTiles + 1u);
         const uint32_t cut_slack =
-            Pu > static_cast<uint32_t>(k) + 132u + kCompactSlack ? kCompactSlack : Pu - static_cast<uint32_t>(k) - 132u;
+            Pu > static_cast<uint32_t>(k) + room + kCompactSlack ? kCompactSlack : Pu - static_cast<uint32_t>(k) - room;
         uint32_t acc_it = 0, w_it = 0;
         bool bad = false;
         for (int64_t r = 0; r * G < U; ++r) {
@@ -951,6 +956,7 @@ __global__ void __launch_bounds__(SelCfg<H, D>::THREADS, 1)
                 }
             };
             if (ui.ntiles > 0) load_w();
+            bool need_acc = false, bad_acc = false;
             for (int j = 0; j < ui.ntiles; ++j) {
                 const uint32_t buf = acc_it & 1u;
                 SI_TR_T0(tf0);
@@ -992,18 +998,24 @@ __global__ void __launch_bounds__(SelCfg<H, D>::THREADS, 1)
                             const uint32_t bal = __ballot_sync(0xffffffffu, pass);
                             if (pass) pool[(half * C::QH + q) * P + bw(q) + cw[q] + __popc(bal & lanemask_lt())] = key;
                             cw[q] += static_cast<uint32_t>(__popc(bal));
-                            need |= cw[q] + 32u > fw(q);
+                            need |= cw[q] + 32u * kCheckTiles > fw(q);
                         }
                     }
                 }
                 SI_TR_T0(tfl0);
-                // One barrier per tile (abort and cut requests are OR-reduced);
-                // two more only when some sub-range is nearly full or a wait failed.
-                const bool bad_here = !ok || *abort_flag;
-                SI_TR_DEPI(static_cast<int>(need));
+                // One barrier every kCheckTiles tiles (abort and cut requests are
+                // OR-reduced; sub-ranges keep room for kCheckTiles tiles of
+                // appends); two more only when some sub-range is nearly full or
+                // a wait failed.
+                need_acc |= need;
+                bad_acc |= !ok;
+                if ((j + 1) % kCheckTiles != 0 && j + 1 != ui.ntiles) continue;
+                const bool bad_here = bad_acc || *abort_flag;
+                SI_TR_DEPI(static_cast<int>(need_acc));
                 SI_TR_ADD(kTrEpiFilter, tfl0, tr_lead);
                 SI_TR_T0(tb0);
-                const bool any_flag = bar_red_or(bar_id, 128, bad_here || need);
+                const bool any_flag = bar_red_or(bar_id, 128, bad_here || need_acc);
+                need_acc = false;
                 SI_TR_ADD(kTrEpiBarrier, tb0, tr_lead);
                 if (any_flag) {
                     SI_TR_T0(tc0);
@@ -1020,7 +1032,8 @@ __global__ void __launch_bounds__(SelCfg<H, D>::THREADS, 1)
                     for (int q = 0; q < C::QH; ++q) {
                         const uint32_t* c4 = cntw[half][q];
                         const uint32_t f = fw(q);
-                        const bool cut = c4[0] + 32u > f || c4[1] + 32u > f || c4[2] + 32u > f || c4[3] + 32u > f;
+                        constexpr uint32_t mg = 32u * kCheckTiles;
+                        const bool cut = c4[0] + mg > f || c4[1] + mg > f || c4[2] + mg > f || c4[3] + mg > f;
                         if (!cut) continue;  // uniform over the half
                         uint64_t* pq = pool + (half * C::QH + q) * P;
                         uint32_t kept = 0;
