@@ -265,14 +265,16 @@ si_status si_sort_topk(int32_t* out_idx, float* out_score, int64_t rows, int k, 
     const unsigned threads = 32 * si::kSortWarps;
     int k2 = 32;
     while (k2 < k) k2 <<= 1;
+    if (rows > 0x7FFFFFFF) return SI_ERR_UNSUPPORTED;
+    const unsigned rows_grid = static_cast<unsigned>(rows);  // one block per row (long rows)
     switch (k2 / 32) {
         case 1: si::sort_rows_kernel<1><<<blocks, threads, 0, s>>>(out_idx, out_score, rows, k); break;
         case 2: si::sort_rows_kernel<2><<<blocks, threads, 0, s>>>(out_idx, out_score, rows, k); break;
         case 4: si::sort_rows_kernel<4><<<blocks, threads, 0, s>>>(out_idx, out_score, rows, k); break;
         case 8: si::sort_rows_kernel<8><<<blocks, threads, 0, s>>>(out_idx, out_score, rows, k); break;
         case 16: si::sort_rows_kernel<16><<<blocks, threads, 0, s>>>(out_idx, out_score, rows, k); break;
-        case 32: si::sort_rows_kernel<32><<<blocks, threads, 0, s>>>(out_idx, out_score, rows, k); break;
-        case 64: si::sort_rows_kernel<64><<<blocks, threads, 0, s>>>(out_idx, out_score, rows, k); break;
+        case 32: si::sort_rows_smem_kernel<1024><<<rows_grid, 512, 0, s>>>(out_idx, out_score, rows, k); break;
+        case 64: si::sort_rows_smem_kernel<2048><<<rows_grid, 1024, 0, s>>>(out_idx, out_score, rows, k); break;
         default: return SI_ERR_UNSUPPORTED;
     }
     return cudaGetLastError() == cudaSuccess ? SI_OK : SI_ERR_CUDA;

@@ -334,9 +334,23 @@ __device__ __forceinline__ uint32_t half_sum(uint32_t c, CutScratch& cs, int tid
 struct StreamKeys {
     const uint64_t* pool;
     PoolRegions rg;
+    // Eight loads in flight per thread: these pools live in global memory.
     template <typename F>
     __device__ __forceinline__ void for_each(int tid, F f) const {
-        half_for_each(pool, rg, tid, f);
+#pragma unroll 1
+        for (int r = 0; r < 5; ++r) {
+            const uint64_t* base = pool + rg.start[r];
+            const int len = rg.len[r];
+            int i = tid;
+            for (; i + 7 * 128 < len; i += 8 * 128) {
+                uint64_t x[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) x[u] = base[i + u * 128];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) f(x[u]);
+            }
+            for (; i < len; i += 128) f(base[i]);
+        }
     }
 };
 
@@ -913,7 +927,7 @@ __global__ void __launch_bounds__(SelCfg<H, D>::THREADS, 1)
             // except the append sub-range: survivors [0, kp), this warp's
             // sub-range [bw, bw + fw) holding cw appended keys, lower bound lb.
             uint64_t lb[C::QH];
-            uint32_t kp[C::QH], cw[C::QH];
+            uint32_t kp[C::QH] = {}, cw[C::QH] = {};
             // free room after the survivors, split four ways: this warp's sub-range
             auto fw = [&](int q) { return (Pu - kp[q]) / 4u; };
             auto bw = [&](int q) { return kp[q] + wih * fw(q); };

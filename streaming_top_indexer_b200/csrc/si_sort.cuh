@@ -71,6 +71,47 @@ __global__ void __launch_bounds__(32 * kSortWarps) sort_rows_kernel(int32_t* __r
     }
 }
 
+// Same ordering for long rows (32*E > 512): one block of K2/2 threads per row
+// runs the bitonic network in shared memory, one compare-exchange per thread
+// and stage, instead of holding 64 keys per lane in registers.
+template <int K2>
+__global__ void __launch_bounds__(K2 / 2) sort_rows_smem_kernel(int32_t* __restrict__ idx, float* __restrict__ score,
+                                                                 int64_t rows, int k) {
+    __shared__ uint64_t v[K2];
+    const int tid = threadIdx.x;
+    const int64_t row = blockIdx.x;
+    if (row >= rows) return;
+    int32_t* ri = idx + row * k;
+    float* rs = score + row * k;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int i = tid + h * (K2 / 2);
+        v[i] = (i < k) ? pack_key(rs[i], static_cast<uint32_t>(ri[i])) : 0ull;
+    }
+    __syncthreads();
+    for (int size = 2; size <= K2; size <<= 1) {
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            const int i = ((tid / stride) * 2 * stride) + (tid % stride);  // lower index of this thread's pair
+            const int j = i + stride;
+            const bool desc = (i & size) == 0;
+            const uint64_t a = v[i], b = v[j];
+            if (desc ? (a < b) : (a > b)) {
+                v[i] = b;
+                v[j] = a;
+            }
+            __syncthreads();
+        }
+    }
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int i = tid + h * (K2 / 2);
+        if (i < k) {
+            ri[i] = key_index(v[i]);
+            rs[i] = key_score(v[i]);
+        }
+    }
+}
+
 // Every row all padding (no key is visible to any query).
 __global__ void pad_rows_kernel(int32_t* __restrict__ idx, float* __restrict__ score, int64_t n) {
     const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
