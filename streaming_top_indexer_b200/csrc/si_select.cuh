@@ -42,13 +42,13 @@ namespace si {
 
 // Optional cycle tracing (build flag SI_TRACE; off in the product library).
 // Every thread accumulates cycle counts in registers; lane 0 of each warp
-// writes them to SelectParams::trace[(cta * 10 + warp) * kTraceSlots + slot].
-constexpr int kTraceSlots = 16;
-constexpr int kTraceWarps = 10;
+// writes them to SelectParams::trace[(cta * kTraceWarps + warp) * kTraceSlots + slot].
+constexpr int kTraceSlots = 20;
+constexpr int kTraceWarps = 12;  // warps per CTA (checked against SelCfg::THREADS)
 enum : int {
     kTrMmaKcFull = 0, kTrMmaAccEmpty, kTrMmaQFull, kTrProdKcEmpty, kTrProdQEmpty, kTrEpiAccFull,
     kTrEpiScores, kTrEpiArrive, kTrEpiFilter, kTrEpiBarrier, kTrEpiCompact, kTrCompactions, kTrTiles,
-    kTrTotal, kTrEpiWFull, kTrEpiFinal
+    kTrTotal, kTrEpiWFull, kTrEpiFinal, kTrEpiAppend, kTrEpiUnit
 };
 #ifdef SI_TRACE
 __device__ __forceinline__ long long tr_clock() {
@@ -107,9 +107,11 @@ struct SelCfg {
     static constexpr int EPI_WARP0 = 4;         // warps 0-3: TMA producer, MMA issuer, two idle
     static constexpr int THREADS = 32 * EPI_WARP0 + 32 * EPI_WARPS;
     // Registers: launched at 168 per thread; the control warpgroup then gives
-    // registers up so that each epilogue thread can hold its 128 head weights.
-    static constexpr uint32_t REGS_LAUNCH = 168, REGS_CTRL = 56, REGS_EPI = 224;
+    // up all but the minimum (24) so that each epilogue thread can hold its
+    // 128 head weights and two TMEM chunks in flight (240).
+    static constexpr uint32_t REGS_LAUNCH = 168, REGS_CTRL = 24, REGS_EPI = 240;
     static_assert(NGROUPS == 2, "register split assumes two epilogue warpgroups");
+    static_assert(THREADS / 32 == kTraceWarps, "trace layout holds one slot row per warp");
     static_assert(REGS_CTRL * 128 + REGS_EPI * 32 * EPI_WARPS == REGS_LAUNCH * THREADS,
                   "the register split must add up to the launch allocation");
     static constexpr uint32_t TMEM_COLS = 512;  // two 256-column accumulators
@@ -129,9 +131,11 @@ struct SelCfg {
     static constexpr uint32_t smem_bytes(bool pool_in_smem, int P) {
         return dyn_bytes(pool_in_smem, P) + STATIC_BYTES;
     }
-    // Epilogue accumulators: NP float2 partial sums per query, so that every
-    // dependent FMA chain is at most 8 long (4 for H_I=8).
-    static constexpr int NP = (8 / QH) < 1 ? 1 : ((8 / QH) > 4 ? 4 : 8 / QH);
+    // Epilogue accumulators: NP float2 partial sums per query (two at H_I=64,
+    // one otherwise).  More partial sums shorten the dependent FMA chains but
+    // cost registers that the epilogue, holding 128 head weights per thread,
+    // does not have: measured, two beat four at H_I=64.
+    static constexpr int NP = (4 / QH) < 1 ? 1 : ((4 / QH) > 2 ? 2 : 4 / QH);
 };
 
 // Extra entries an intermediate pool cut may keep above k (the cut at the end
@@ -923,6 +927,7 @@ __global__ void __launch_bounds__(SelCfg<H, D>::THREADS, 1)
             const int64_t u = unit_of_round(r, G, cta);
             if (u >= U) continue;
             const UnitInfo ui = decode_unit(u, p, C::QT);
+            SI_TR_T0(tun0);
             // Pool state of each query of the half, identical in the four warps
             // except the append sub-range: survivors [0, kp), this warp's
             // sub-range [bw, bw + fw) holding cw appended keys, lower bound lb.
@@ -970,6 +975,7 @@ __global__ void __launch_bounds__(SelCfg<H, D>::THREADS, 1)
                 }
             };
             if (ui.ntiles > 0) load_w();
+            SI_TR_ADD(kTrEpiUnit, tun0, tr_lead);
             bool need_acc = false, bad_acc = false;
             for (int j = 0; j < ui.ntiles; ++j) {
                 const uint32_t buf = acc_it & 1u;
@@ -991,6 +997,7 @@ __global__ void __launch_bounds__(SelCfg<H, D>::THREADS, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar(kBarAccEmpty + buf));
                 SI_TR_ADD(kTrEpiArrive, tar0, tr_lead);
+                SI_TR_T0(tap0);
                 const int32_t s = j * C::BM + quarter * 32 + lane;
                 bool need = false;
                 if (ok) {
@@ -1016,6 +1023,7 @@ __global__ void __launch_bounds__(SelCfg<H, D>::THREADS, 1)
                         }
                     }
                 }
+                SI_TR_ADD(kTrEpiAppend, tap0, tr_lead);
                 SI_TR_T0(tfl0);
                 // One barrier every kCheckTiles tiles (abort and cut requests are
                 // OR-reduced; sub-ranges keep room for kCheckTiles tiles of
