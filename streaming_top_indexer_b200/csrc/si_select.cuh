@@ -286,13 +286,18 @@ struct PoolRegions {
     __device__ __forceinline__ int total() const { return len[0] + len[1] + len[2] + len[3] + len[4]; }
 };
 
+// Most keys an exact cut gathers between two adjacent samples.
+constexpr int kCandCap = 256;
+
 // Per-half scratch of a pool cut, in shared memory.
 struct CutScratch {
-    unsigned long long srt[32];   // 32 samples sorted descending; 0 (below any key) past the last
-    unsigned long long cand[64];  // keys between two adjacent samples (exact cut)
-    unsigned long long xch[8];    // cross-warp exchange
-    uint32_t hist[256];           // radix fallback histogram
-    uint32_t rcnt[2][4];          // per-warp counts, double-buffered by call parity
+    unsigned long long srt[32];  // 32 samples sorted descending; 0 (below any key) past the last
+    union {
+        unsigned long long cand[kCandCap];  // staged samples, then the keys of the bracket (exact cut)
+        uint32_t hist[256];                 // radix fallback histogram
+    };
+    unsigned long long xch[8];   // cross-warp exchange
+    uint32_t rcnt[2][4];         // per-warp counts, double-buffered by call parity
     uint32_t ncand;
 };
 
@@ -309,13 +314,18 @@ __device__ __forceinline__ void half_for_each(const uint64_t* pool, const PoolRe
     }
 }
 
-// Address of virtual position v of the address-ordered regions (v < total).
+// Address of virtual position v of the address-ordered regions (v < total):
+// region r holds positions [e_r, e_r + len_r) with e_r the sum of the
+// earlier lengths, and the last region whose e_r <= v holds v (an empty
+// region ends where it starts).  The e_r are the same for every v, so a run
+// of calls shares them and each call is four independent compare-selects.
 __device__ __forceinline__ int region_addr(const PoolRegions& rg, int v) {
-    int a = -1;
+    int a = rg.start[0] + v;
+    int e = rg.len[0];
 #pragma unroll
-    for (int r = 0; r < 5; ++r) {
-        if (a < 0 && v < rg.len[r]) a = rg.start[r] + v;
-        v -= rg.len[r];
+    for (int r = 1; r < 5; ++r) {
+        a = v >= e ? rg.start[r] + (v - e) : a;
+        e += rg.len[r];
     }
     return a;
 }
@@ -386,39 +396,6 @@ __device__ __forceinline__ uint32_t half_count_ge(const Keys& keys, uint64_t L, 
     uint32_t c = 0;
     keys.for_each(tid, [&](uint64_t x) { c += x >= L ? 1u : 0u; });
     return half_sum(c, cs, tid, bar_id, phase);
-}
-
-// Warp-wide bitonic sort, descending, of 32*E keys: element i is v[i/32] of lane i%32.
-template <int E>
-__device__ __forceinline__ void warp_sort_desc(uint64_t (&v)[E], int lane) {
-#pragma unroll
-    for (int size = 2; size <= 32 * E; size <<= 1) {
-#pragma unroll
-        for (int stride = size >> 1; stride > 0; stride >>= 1) {
-            if (stride >= 32) {
-                const int es = stride >> 5;
-#pragma unroll
-                for (int e = 0; e < E; ++e) {
-                    const int pe = e ^ es;
-                    if (pe > e) {
-                        const bool desc = ((e * 32) & size) == 0;
-                        const uint64_t a = v[e], b = v[pe];
-                        const bool sw = desc ? (a < b) : (a > b);
-                        v[e] = sw ? b : a;
-                        v[pe] = sw ? a : b;
-                    }
-                }
-            } else {
-#pragma unroll
-                for (int e = 0; e < E; ++e) {
-                    const int i = e * 32 + lane;
-                    const uint64_t o = __shfl_xor_sync(0xffffffffu, v[e], stride);
-                    const bool take_max = ((lane & stride) == 0) == ((i & size) == 0);
-                    v[e] = take_max ? (v[e] > o ? v[e] : o) : (v[e] < o ? v[e] : o);
-                }
-            }
-        }
-    }
 }
 
 // Radix select (fallback): lower bound L with k <= #(keys >= L) <= k + slack,
@@ -514,13 +491,16 @@ __device__ __noinline__ uint64_t half_radix_bound(const uint64_t* pool, const Po
 // Lower bound L of the best keys in the regions, by the 128 threads of one
 // epilogue half: k <= #(keys >= L) <= max_keep (max_keep == k: exactly the k
 // best).  Needs n > k.
-//  1. Warp 0 draws 32 evenly spaced keys and sorts them in registers.
+//  1. Warp 0 draws 32 evenly spaced keys and places each at its rank among
+//     them (keys are distinct), which sorts them.
 //  2. Counting passes (one barrier each) test samples near the rank that
 //     predicts the target count, stepping one sample at a time, until a
 //     sample qualifies or two adjacent samples bracket the k-th key.
-//  3. Exact cut: the keys between the bracketing samples (about n/32) are
-//     gathered and one warp sorts them to pick the k-th.
-//  4. A bracket holding more than 64 keys falls back to the radix select.
+//  3. Exact cut: the keys between the bracketing samples (about n/16 for the
+//     bracket that holds a given rank) are gathered, and each is ranked
+//     against the others by the whole half to pick the k-th.
+//  4. A bracket holding more than kCandCap keys falls back to the radix
+//     select.
 template <typename Keys>
 __device__ __forceinline__ uint64_t half_select_bound(const Keys& keys, const uint64_t* pool, const PoolRegions& rg,
                                                       int k, uint32_t max_keep, CutScratch& cs, int tid,
@@ -529,10 +509,17 @@ __device__ __forceinline__ uint64_t half_select_bound(const Keys& keys, const ui
     const int n = rg.total();
     const int ns = n < 32 ? n : 32;
     if (tid < 32) {
-        uint64_t v[1];
-        v[0] = lane < ns ? pool[region_addr(rg, n >= 32 ? (lane * n) >> 5 : lane)] : 0ull;
-        warp_sort_desc<1>(v, lane);
-        cs.srt[lane] = v[0];
+        // Samples are distinct keys; each is placed at its rank among them.
+        const uint64_t me = lane < ns ? pool[region_addr(rg, n >= 32 ? (lane * n) >> 5 : lane)] : 0ull;
+        cs.cand[lane] = me;
+        __syncwarp();
+        int r = lane;
+        if (lane < ns) {
+            r = 0;
+#pragma unroll 8
+            for (int i = 0; i < 32; ++i) r += cs.cand[i] > me ? 1 : 0;
+        }
+        cs.srt[r] = me;
     }
     if (tid == 0) cs.ncand = 0;
     bar_sync(bar_id, 128);
@@ -558,7 +545,7 @@ __device__ __forceinline__ uint64_t half_select_bound(const Keys& keys, const ui
         if (r <= lo_r || r >= hi_r) break;
     }
     const uint32_t m = c_hi - c_lo;  // keys in [lower, upper)
-    if (hi_r - lo_r != 1 || m > 64u) {
+    if (hi_r - lo_r != 1 || m > static_cast<uint32_t>(kCandCap)) {
         bar_sync(bar_id, 128);
         return half_radix_bound(pool, rg, k, max_keep - ku, cs, tid, bar_id);
     }
@@ -568,14 +555,16 @@ __device__ __forceinline__ uint64_t half_select_bound(const Keys& keys, const ui
         if (x >= lower && x < upper) cs.cand[atomicAdd(&cs.ncand, 1u)] = x;
     });
     bar_sync(bar_id, 128);
-    if (tid < 32) {
-        uint64_t v[2];
-        v[0] = lane < static_cast<int>(m) ? cs.cand[lane] : 0ull;
-        v[1] = lane + 32 < static_cast<int>(m) ? cs.cand[lane + 32] : 0ull;
-        warp_sort_desc<2>(v, lane);
-        const int want = static_cast<int>(ku - c_lo) - 1;  // 0-based rank inside the bracket
-        if (lane == want) cs.xch[0] = v[0];
-        if (lane + 32 == want) cs.xch[0] = v[1];
+    // The bracket's keys are distinct: the one with exactly `want` keys of the
+    // bracket above it is the k-th key.
+    const int want = static_cast<int>(ku - c_lo) - 1;  // 0-based rank inside the bracket
+    const int mi = static_cast<int>(m);
+    for (int c = tid; c < mi; c += 128) {
+        const uint64_t x = cs.cand[c];
+        int r = 0;
+#pragma unroll 8
+        for (int i = 0; i < mi; ++i) r += cs.cand[i] > x ? 1 : 0;
+        if (r == want) cs.xch[0] = x;
     }
     bar_sync(bar_id, 128);
     return cs.xch[0];
