@@ -330,12 +330,27 @@ __device__ __forceinline__ int region_addr(const PoolRegions& rg, int v) {
     return a;
 }
 
+// Exclusive prefix over the warp of per-lane counts below 32, and the warp's
+// total: bit b of every lane's count is one ballot, so the five ballots and
+// population counts are independent of one another.
+__device__ __forceinline__ uint32_t warp_prefix_small(uint32_t v, int lane, uint32_t& total) {
+    const uint32_t below = (1u << lane) - 1u;
+    uint32_t pre = 0, tot = 0;
+#pragma unroll
+    for (int b = 0; b < 5; ++b) {
+        const uint32_t m = __ballot_sync(0xffffffffu, (v >> b) & 1u);
+        pre += static_cast<uint32_t>(__popc(m & below)) << b;
+        tot += static_cast<uint32_t>(__popc(m)) << b;
+    }
+    total = tot;
+    return pre;
+}
+
 // Sum over the 128 threads of the half, with one barrier; `phase` selects the
 // exchange buffer and must advance identically in every thread.
 __device__ __forceinline__ uint32_t half_sum(uint32_t c, CutScratch& cs, int tid, uint32_t bar_id, uint32_t& phase) {
     const int lane = tid & 31, wq = tid >> 5;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+    c = __reduce_add_sync(0xffffffffu, c);
     uint32_t* rc = cs.rcnt[phase & 1u];
     ++phase;
     if (lane == 0) rc[wq] = c;
@@ -369,6 +384,7 @@ struct StreamKeys {
 };
 
 constexpr int kRegKeys = 16;
+static_assert(kRegKeys < 32, "walk prefix counts fit in five bits");
 
 struct RegKeys {
     uint64_t x[kRegKeys];
@@ -580,7 +596,7 @@ template <typename Emit>
 __device__ __forceinline__ uint32_t half_walk_kept(const uint64_t* pool, const PoolRegions& rg, uint64_t L,
                                                    CutScratch& cs, int tid, uint32_t bar_id, uint32_t& phase,
                                                    Emit emit) {
-    constexpr int EP = 16;  // entries per thread per chunk
+    constexpr int EP = 16;  // entries per thread per chunk (the walk prefix needs EP < 32)
     const int lane = tid & 31, wq = tid >> 5;
     const int n = rg.total();
     uint32_t out = 0;
@@ -595,19 +611,14 @@ __device__ __forceinline__ uint32_t half_walk_kept(const uint64_t* pool, const P
             keep |= (kp ? 1u : 0u) << j;
             mine += kp ? 1u : 0u;
         }
-        // exclusive prefix of `mine` over the warp, and per-warp totals
-        uint32_t incl = mine;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += t;
-        }
-        const uint32_t wtot = __shfl_sync(0xffffffffu, incl, 31);
+        // exclusive prefix of `mine` (at most EP < 32) over the warp, and per-warp totals
+        uint32_t wtot;
+        const uint32_t excl = warp_prefix_small(mine, lane, wtot);
         uint32_t* rc = cs.rcnt[phase & 1u];
         ++phase;
         if (lane == 0) rc[wq] = wtot;
         bar_sync(bar_id, 128);
-        uint32_t pos = out + incl - mine, total = 0;
+        uint32_t pos = out + excl, total = 0;
 #pragma unroll
         for (int w = 0; w < 4; ++w) {
             const uint32_t cw = rc[w];
@@ -635,18 +646,13 @@ __device__ __forceinline__ uint32_t half_walk_reg(const RegKeys& rk, uint64_t L,
         keep |= (kp ? 1u : 0u) << j;
         mine += kp ? 1u : 0u;
     }
-    uint32_t incl = mine;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += t;
-    }
-    const uint32_t wtot = __shfl_sync(0xffffffffu, incl, 31);
+    uint32_t wtot;
+    const uint32_t excl = warp_prefix_small(mine, lane, wtot);  // mine <= kRegKeys < 32
     uint32_t* rc = cs.rcnt[phase & 1u];
     ++phase;
     if (lane == 0) rc[wq] = wtot;
     bar_sync(bar_id, 128);
-    uint32_t pos = incl - mine, total = 0;
+    uint32_t pos = excl, total = 0;
 #pragma unroll
     for (int w = 0; w < 4; ++w) {
         const uint32_t cw = rc[w];
