@@ -51,7 +51,8 @@ uint32_t select_smem(int H, int D, bool pool_in_smem, int P) {
 // Where the per-query candidate pools live and how large they are.  A pool
 // holds at least max(2k, k+288) entries (room for k + 28 survivors of a cut
 // plus two tiles of appends in each warp's sub-range); in shared memory it takes all the
-// room left (fewer pool cuts), otherwise 4k entries in the workspace.
+// room left (fewer pool cuts), otherwise 4k entries in the workspace, and
+// the shared memory they leave holds the exact-cut candidate buffers.
 struct PoolPlan {
     bool smem;
     int P;
@@ -61,7 +62,7 @@ PoolPlan pool_plan(int H, int D, int k) {
     auto r32 = [](int x) { return (x + 31) / 32 * 32; };
     const int min_p = r32(2 * k > k + 288 ? 2 * k : k + 288);
     const uint32_t qt = 256u / static_cast<uint32_t>(H);
-    const uint32_t fixed = select_smem(H, D, false, 0);
+    const uint32_t fixed = select_smem(H, D, true, 0);  // everything but the pools
     if (fixed + qt * static_cast<uint32_t>(min_p) * 8u <= kMaxDynSmem) {
         int p = static_cast<int>((kMaxDynSmem - fixed) / (qt * 8u)) / 32 * 32;
         if (p > 65504) p = 65504;  // pool counts are 16-bit fields

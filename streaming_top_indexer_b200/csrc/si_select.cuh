@@ -125,8 +125,13 @@ struct SelCfg {
     // Upper bound of the kernel's static shared memory (the host checks the
     // real figure at launch; pools in shared memory are sized with this).
     static constexpr uint32_t STATIC_BYTES = 6144;
+    // With the pools in the workspace, each epilogue group gets a buffer of
+    // STREAM_CAND keys in shared memory for the exact cut of its large pools.
+    static constexpr int STREAM_CAND = 3072;
     static constexpr uint32_t dyn_bytes(bool pool_in_smem, int P) {
-        return OFF_POOL + (pool_in_smem ? static_cast<uint32_t>(QT) * P * 8u : 0u) + ALIGN_SLACK;
+        return OFF_POOL +
+               (pool_in_smem ? static_cast<uint32_t>(QT) * P * 8u : static_cast<uint32_t>(NGROUPS * STREAM_CAND) * 8u) +
+               ALIGN_SLACK;
     }
     static constexpr uint32_t smem_bytes(bool pool_in_smem, int P) {
         return dyn_bytes(pool_in_smem, P) + STATIC_BYTES;
@@ -515,12 +520,15 @@ __device__ __noinline__ uint64_t half_radix_bound(const uint64_t* pool, const Po
 //  3. Exact cut: the keys between the bracketing samples (about n/16 for the
 //     bracket that holds a given rank) are gathered, and each is ranked
 //     against the others by the whole half to pick the k-th.
-//  4. A bracket holding more than kCandCap keys falls back to the radix
-//     select.
-template <typename Keys>
+//  4. With BIG (pools in the workspace), a bracket of more than kCandCap
+//     keys is gathered into `big` (up to big_cap keys, shared memory) and
+//     the same select picks the k-th key among them.  Any larger bracket
+//     falls back to the radix select.
+template <bool BIG = false, typename Keys>
 __device__ __forceinline__ uint64_t half_select_bound(const Keys& keys, const uint64_t* pool, const PoolRegions& rg,
                                                       int k, uint32_t max_keep, CutScratch& cs, int tid,
-                                                      uint32_t bar_id, uint32_t& phase) {
+                                                      uint32_t bar_id, uint32_t& phase, uint64_t* big = nullptr,
+                                                      int big_cap = 0) {
     const int lane = tid & 31;
     const int n = rg.total();
     const int ns = n < 32 ? n : 32;
@@ -561,16 +569,42 @@ __device__ __forceinline__ uint64_t half_select_bound(const Keys& keys, const ui
         if (r <= lo_r || r >= hi_r) break;
     }
     const uint32_t m = c_hi - c_lo;  // keys in [lower, upper)
-    if (hi_r - lo_r != 1 || m > static_cast<uint32_t>(kCandCap)) {
+    const bool small = m <= static_cast<uint32_t>(kCandCap);
+    bool use_big = false;
+    if constexpr (BIG) use_big = !small && m <= static_cast<uint32_t>(big_cap);
+    if (hi_r - lo_r != 1 || !(small || use_big)) {
         bar_sync(bar_id, 128);
         return half_radix_bound(pool, rg, k, max_keep - ku, cs, tid, bar_id);
     }
     const uint64_t upper = lo_r >= 0 ? cs.srt[lo_r] : ~0ull;
     const uint64_t lower = hi_r < ns ? cs.srt[hi_r] : 0ull;
+    uint64_t* dst = use_big ? big : reinterpret_cast<uint64_t*>(cs.cand);
     keys.for_each(tid, [&](uint64_t x) {
-        if (x >= lower && x < upper) cs.cand[atomicAdd(&cs.ncand, 1u)] = x;
+        if (x >= lower && x < upper) dst[atomicAdd(&cs.ncand, 1u)] = x;
     });
     bar_sync(bar_id, 128);
+    if constexpr (BIG) {
+        if (use_big) {
+            // The k-th key is the (k - c_lo)-th of the bracket (fewer than m,
+            // since no sample qualified): the same select over the buffer.
+            PoolRegions one;
+            one.start[0] = 0;
+            one.len[0] = static_cast<int>(m);
+#pragma unroll
+            for (int r2 = 1; r2 < 5; ++r2) {
+                one.start[r2] = static_cast<int>(m);
+                one.len[r2] = 0;
+            }
+            const int kb = static_cast<int>(ku - c_lo);
+            if (m <= 128u * kRegKeys) {
+                RegKeys rk;
+                rk.load(big, one, tid);
+                return half_select_bound(rk, big, one, kb, static_cast<uint32_t>(kb), cs, tid, bar_id, phase);
+            }
+            const StreamKeys sk{big, one};
+            return half_select_bound(sk, big, one, kb, static_cast<uint32_t>(kb), cs, tid, bar_id, phase);
+        }
+    }
     // The bracket's keys are distinct: the one with exactly `want` keys of the
     // bracket above it is the k-th key.
     const int want = static_cast<int>(ku - c_lo) - 1;  // 0-based rank inside the bracket
@@ -668,18 +702,24 @@ __device__ __forceinline__ uint32_t half_walk_reg(const RegKeys& rk, uint64_t L,
 // Cuts one query's pool to its best keys -- between k and max_keep of them,
 // or all when there are at most k -- packed at the front of the pool, by the
 // 128 threads of the half.  Returns the new lower bound; `kept` gets the count.
+// `big`: the group's shared-memory candidate buffer (STREAM_CAND keys) when
+// the pools are in the workspace, else null.
 __device__ __noinline__ uint64_t cut_pool(uint64_t* pq, PoolRegions rg, int k, uint32_t max_keep, uint64_t lb,
                                           CutScratch& cs, int tid, uint32_t bar_id, uint32_t& phase,
-                                          uint32_t& kept) {
+                                          uint32_t& kept, uint64_t* big, int big_cap) {
     uint64_t L = lb;
     if (rg.total() <= 128 * kRegKeys) {
         RegKeys rk;
         rk.load(pq, rg, tid);
-        if (rk.n > k) L = half_select_bound(rk, pq, rg, k, max_keep, cs, tid, bar_id, phase);
+        if (rk.n > k)
+            L = big ? half_select_bound<true>(rk, pq, rg, k, max_keep, cs, tid, bar_id, phase, big, big_cap)
+                    : half_select_bound(rk, pq, rg, k, max_keep, cs, tid, bar_id, phase);
         kept = half_walk_reg(rk, L, cs, tid, bar_id, phase, [&](uint64_t x, uint32_t pos) { pq[pos] = x; });
     } else {
         const StreamKeys sk{pq, rg};
-        if (rg.total() > k) L = half_select_bound(sk, pq, rg, k, max_keep, cs, tid, bar_id, phase);
+        if (rg.total() > k)
+            L = big ? half_select_bound<true>(sk, pq, rg, k, max_keep, cs, tid, bar_id, phase, big, big_cap)
+                    : half_select_bound(sk, pq, rg, k, max_keep, cs, tid, bar_id, phase);
         kept = half_walk_kept(pq, rg, L, cs, tid, bar_id, phase, [&](uint64_t x, uint32_t pos) { pq[pos] = x; });
     }
     return L;
@@ -688,7 +728,8 @@ __device__ __noinline__ uint64_t cut_pool(uint64_t* pq, PoolRegions rg, int k, u
 // Writes the k best keys of one query's pool (or all, when fewer), unordered,
 // to its output row, then pads the row with (-1, -inf); by the half.
 __device__ __noinline__ void emit_best(const uint64_t* pq, PoolRegions rg, int k, CutScratch& cs, int tid,
-                                       uint32_t bar_id, uint32_t& phase, int32_t* out_idx, float* out_score) {
+                                       uint32_t bar_id, uint32_t& phase, int32_t* out_idx, float* out_score,
+                                       uint64_t* big, int big_cap) {
     auto emit = [&](uint64_t x, uint32_t pos) {
         out_idx[pos] = key_index(x);
         out_score[pos] = key_score(x);
@@ -697,13 +738,19 @@ __device__ __noinline__ void emit_best(const uint64_t* pq, PoolRegions rg, int k
     if (rg.total() <= 128 * kRegKeys) {
         RegKeys rk;
         rk.load(pq, rg, tid);
-        const uint64_t L = rk.n > k ? half_select_bound(rk, pq, rg, k, static_cast<uint32_t>(k), cs, tid, bar_id, phase)
-                                    : 0ull;
+        const uint32_t ku = static_cast<uint32_t>(k);
+        const uint64_t L =
+            rk.n <= k ? 0ull
+            : big     ? half_select_bound<true>(rk, pq, rg, k, ku, cs, tid, bar_id, phase, big, big_cap)
+                      : half_select_bound(rk, pq, rg, k, ku, cs, tid, bar_id, phase);
         out = half_walk_reg(rk, L, cs, tid, bar_id, phase, emit);
     } else {
         const StreamKeys sk{pq, rg};
+        const uint32_t ku = static_cast<uint32_t>(k);
         const uint64_t L =
-            rg.total() > k ? half_select_bound(sk, pq, rg, k, static_cast<uint32_t>(k), cs, tid, bar_id, phase) : 0ull;
+            rg.total() <= k ? 0ull
+            : big           ? half_select_bound<true>(sk, pq, rg, k, ku, cs, tid, bar_id, phase, big, big_cap)
+                            : half_select_bound(sk, pq, rg, k, ku, cs, tid, bar_id, phase);
         out = half_walk_kept(pq, rg, L, cs, tid, bar_id, phase, emit);
     }
     for (int i = static_cast<int>(out) + tid; i < k; i += 128) {
@@ -907,6 +954,8 @@ __global__ void __launch_bounds__(SelCfg<H, D>::THREADS, 1)
         const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
         const int htid = wih * 32 + lane;  // thread index within the half
         CutScratch& cs = cut_s[half];
+        // workspace pools: the group's exact-cut buffer takes the room of the shared-memory pools
+        uint64_t* big = SMEM_POOL ? nullptr : reinterpret_cast<uint64_t*>(smem + C::OFF_POOL) + half * C::STREAM_CAND;
         uint32_t cphase = 0;  // exchange-buffer parity of the half's cut helpers
         const bool dense = p.dense != nullptr;
         const int k = p.k;
@@ -1056,7 +1105,7 @@ __global__ void __launch_bounds__(SelCfg<H, D>::THREADS, 1)
                         uint32_t kept = 0;
                         const uint64_t L = cut_pool(pq, pool_regions(kp[q], f, c4), k,
                                                     static_cast<uint32_t>(k) + cut_slack, lb[q], cs, htid, bar_id,
-                                                    cphase, kept);
+                                                    cphase, kept, big, C::STREAM_CAND);
                         SI_TR_INC(kTrCompactions, true);
                         kp[q] = kept;
                         lb[q] = L;
@@ -1085,7 +1134,7 @@ __global__ void __launch_bounds__(SelCfg<H, D>::THREADS, 1)
                     if (t >= p.S) continue;  // uniform over the half
                     const int64_t row = (ui.b * p.S + t) * static_cast<int64_t>(k);
                     emit_best(pool + qi * P, pool_regions(kp[q], fw(q), cntw[half][q]), k, cs, htid, bar_id, cphase,
-                              p.out_idx + row, p.out_score + row);
+                              p.out_idx + row, p.out_score + row, big, C::STREAM_CAND);
                     bar_sync(bar_id, 128);
                 }
             }
