@@ -71,43 +71,75 @@ __global__ void __launch_bounds__(32 * kSortWarps) sort_rows_kernel(int32_t* __r
     }
 }
 
-// Same ordering for long rows (32*E > 512): one block of K2/2 threads per row
-// runs the bitonic network in shared memory, one compare-exchange per thread
-// and stage, instead of holding 64 keys per lane in registers.
+// Same ordering for long rows (K2 = 1024 or 2048 keys): one block of K2/8
+// threads per row, eight keys per thread; element i is slot i%8 of thread
+// i/8, so each thread loads and stores 8 consecutive entries.  Partner
+// distances below 8 are register swaps, those below 256 lane shuffles inside
+// the warp, and only the stages at 256 and above (3 for 1024, 6 for 2048)
+// exchange through shared memory, double-buffered with one barrier each.
 template <int K2>
-__global__ void __launch_bounds__(K2 / 2) sort_rows_smem_kernel(int32_t* __restrict__ idx, float* __restrict__ score,
-                                                                 int64_t rows, int k) {
-    __shared__ uint64_t v[K2];
+__global__ void __launch_bounds__(K2 / 8) sort_rows_block_kernel(int32_t* __restrict__ idx,
+                                                                 float* __restrict__ score, int64_t rows, int k) {
+    constexpr int E = 8;
+    __shared__ uint64_t xs[2][K2];
     const int tid = threadIdx.x;
     const int64_t row = blockIdx.x;
     if (row >= rows) return;
     int32_t* ri = idx + row * k;
     float* rs = score + row * k;
+    uint64_t v[E];
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        const int i = tid + h * (K2 / 2);
-        v[i] = (i < k) ? pack_key(rs[i], static_cast<uint32_t>(ri[i])) : 0ull;
+    for (int e = 0; e < E; ++e) {
+        const int i = tid * E + e;
+        v[e] = (i < k) ? pack_key(rs[i], static_cast<uint32_t>(ri[i])) : 0ull;
     }
-    __syncthreads();
+    int buf = 0;
+#pragma unroll
     for (int size = 2; size <= K2; size <<= 1) {
+#pragma unroll
         for (int stride = size >> 1; stride > 0; stride >>= 1) {
-            const int i = ((tid / stride) * 2 * stride) + (tid % stride);  // lower index of this thread's pair
-            const int j = i + stride;
-            const bool desc = (i & size) == 0;
-            const uint64_t a = v[i], b = v[j];
-            if (desc ? (a < b) : (a > b)) {
-                v[i] = b;
-                v[j] = a;
+            if (stride < E) {
+#pragma unroll
+                for (int e = 0; e < E; ++e) {
+                    const int pe = e ^ stride;
+                    if (pe > e) {
+                        const bool desc = ((tid * E + e) & size) == 0;
+                        const uint64_t a = v[e], b = v[pe];
+                        const bool sw = desc ? (a < b) : (a > b);
+                        v[e] = sw ? b : a;
+                        v[pe] = sw ? a : b;
+                    }
+                }
+            } else {
+                const int pt = stride / E;  // partner thread distance
+                const bool lower = (tid & pt) == 0;
+                uint64_t o[E];
+                if (stride < 32 * E) {
+#pragma unroll
+                    for (int e = 0; e < E; ++e) o[e] = __shfl_xor_sync(0xffffffffu, v[e], pt);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < E; ++e) xs[buf][tid * E + e] = v[e];
+                    __syncthreads();
+#pragma unroll
+                    for (int e = 0; e < E; ++e) o[e] = xs[buf][(tid ^ pt) * E + e];
+                    buf ^= 1;
+                }
+#pragma unroll
+                for (int e = 0; e < E; ++e) {
+                    const bool desc = ((tid * E + e) & size) == 0;
+                    const bool take_max = (lower == desc);
+                    v[e] = take_max ? (v[e] > o[e] ? v[e] : o[e]) : (v[e] < o[e] ? v[e] : o[e]);
+                }
             }
-            __syncthreads();
         }
     }
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        const int i = tid + h * (K2 / 2);
+    for (int e = 0; e < E; ++e) {
+        const int i = tid * E + e;
         if (i < k) {
-            ri[i] = key_index(v[i]);
-            rs[i] = key_score(v[i]);
+            ri[i] = key_index(v[e]);
+            rs[i] = key_score(v[e]);
         }
     }
 }
