@@ -2,6 +2,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload long] [--no-e2e] [--no-cpu-baseline]
+    python bench.py --sweep k|s [--workload v4flash] [--sweep-values ...]
 
 A step is one indexer call over one batch of synthetic inputs: the fused
 scoring + selection kernel and the per-row sort (what si_indexer_topk
@@ -13,6 +14,7 @@ Rank 0 prints one JSON line.  `value` is the indexer TFLOP/s of the whole
 job (2*H_I*d_I FLOPs per causally visible query-key pair, all ranks) over
 the device-timed region (max over ranks).  `--impl reference` times the CPU
 oracle (fp64, OpenMP) on bounded row samples of the same workload instead.
+`--sweep k|s` prints one line per design-space cell instead (see run_sweep).
 """
 from __future__ import annotations
 
@@ -337,6 +339,95 @@ def run_ours(args, world, rank, local):
         print(json.dumps(line), flush=True)
 
 
+def materialised_topk_rows(dense, rows, m, k):
+    """Top-k of the given query rows from dense [S,T] scores (NaN where not
+    visible): score descending, index ascending (stable sort), visible only."""
+    T = dense.shape[-1]
+    sub = dense[rows]
+    sub = torch.where(torch.isnan(sub), torch.full_like(sub, float("-inf")), sub)
+    order = torch.sort(-sub, dim=-1, stable=True).indices[:, :min(k, T)]
+    vis = torch.clamp((rows + 1) // m, max=T)
+    return order, vis
+
+
+def run_sweep(args):
+    """Design-space sweep (one GPU): indexer TFLOP/s of select + sort per cell,
+    and recall of each cell's top-k against the materialised baseline (dense
+    scores of the same pipeline, stable-sorted by torch) on sampled rows.  One
+    JSON line per cell.  The cells vary k (--sweep k) or S with T = S/m
+    (--sweep s); queries per unit (256/H_I) and keys per tile (128) are fixed
+    by the tcgen05 tile shape."""
+    import streaming_top_indexer_b200 as si
+    from streaming_top_indexer_b200 import build as sbuild
+    from streaming_top_indexer_b200 import synth
+
+    if sbuild.needs_build():
+        sbuild.build()
+    dev = torch.device("cuda:0")
+    base = synth.WORKLOADS[args.workload]
+    if args.sweep == "k":
+        cells = [(base.S, int(v)) for v in args.sweep_values.split(",")] if args.sweep_values else \
+            [(base.S, v) for v in (64, 128, 256, 512, 1024, 2048)]
+    else:
+        cells = [(int(v), base.k) for v in args.sweep_values.split(",")] if args.sweep_values else \
+            [(v, base.k) for v in (16384, 32768, 65536, 131072, 262144)]
+    stream = torch.cuda.current_stream(dev)
+    dense_cache = {}
+    for S, k in cells:
+        wl = synth.Workload(f"{base.name}-sweep", base.B, S, base.m, base.H, base.D, k, base.kind)
+        B, T, H, D, m = wl.B, wl.T, wl.H, wl.D, wl.m
+        if S not in dense_cache:
+            dense_cache.clear()
+            q, w, kc = synth.generate(wl, seed=args.seed, device=dev)
+            dense = si.indexer_scores(q, w, kc, m)[0] if S * T * 4 <= args.sweep_dense_bytes else None
+            dense_cache[S] = (q, w, kc, dense)
+        q, w, kc, dense = dense_cache[S]
+        idx = torch.empty((B, S, k), dtype=torch.int32, device=dev)
+        sc = torch.empty((B, S, k), dtype=torch.float32, device=dev)
+        ws = torch.zeros(si.workspace_bytes(B, S, T, H, D, m, k), dtype=torch.uint8, device=dev)
+        for _ in range(args.warmup):
+            si.select_topk(q, w, kc, m, k, idx, sc, ws, stream)
+            si.sort_topk(idx, sc, stream)
+        torch.cuda.synchronize(dev)
+        e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        sel, srt = [], []
+        for _ in range(args.steps):
+            e0.record(stream)
+            si.select_topk(q, w, kc, m, k, idx, sc, ws, stream)
+            e1.record(stream)
+            si.sort_topk(idx, sc, stream)
+            e2.record(stream)
+            torch.cuda.synchronize(dev)
+            sel.append(e0.elapsed_time(e1))
+            srt.append(e1.elapsed_time(e2))
+        assert si.check_device_status(ws) == 0, "device error in the sweep"
+        flops = 2.0 * H * D * visible_pairs(B, S, T, m)
+        ms = statistics.median(sel) + statistics.median(srt)
+        cell = {"sweep": args.sweep, "workload": base.name, "B": B, "S": S, "T": T, "H_I": H, "d_I": D, "m": m,
+                "k": k, "value": flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "select_ms": statistics.median(sel),
+                "sort_ms": statistics.median(srt), "steps": args.steps, "warmup": args.warmup,
+                "recall_vs_materialised": None}
+        if dense is not None:
+            g = torch.Generator().manual_seed(args.seed + 1)
+            rows = torch.randperm(S, generator=g)[:args.sweep_rows].to(dev)
+            order, vis = materialised_topk_rows(dense, rows, m, k)
+            got = idx[0, rows].long()
+            rec, exact = [], 0
+            for r in range(rows.numel()):
+                n = int(min(k, int(vis[r])))
+                if n == 0:
+                    continue
+                a = set(order[r, :n].tolist())
+                b = set(got[r, :n].tolist())
+                rec.append(len(a & b) / n)
+                exact += int(torch.equal(order[r, :n], got[r, :n]))
+            cell["recall_vs_materialised"] = {"rows": len(rec), "mean": float(np.mean(rec)) if rec else None,
+                                              "min": float(np.min(rec)) if rec else None,
+                                              "rows_identical": exact}
+        print(json.dumps(cell), flush=True)
+        del idx, sc, ws
+
+
 def e2e_measure(si, q, w, kc, wl, args, world, dev, stream, flops_rank):
     """Same metric through indexer_topk_host: pinned host inputs copied in,
     outputs copied out, inside the timed region every step."""
@@ -377,7 +468,18 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work")
     ap.add_argument("--ref-budget", type=float, default=60.0, help="seconds of oracle work, reference arm")
+    ap.add_argument("--sweep", choices=["k", "s"], default=None,
+                    help="design-space sweep over k or S (one GPU; one JSON line per cell)")
+    ap.add_argument("--sweep-values", default="", help="comma-separated k or S values of the sweep")
+    ap.add_argument("--sweep-rows", type=int, default=256, help="rows checked against the materialised top-k")
+    ap.add_argument("--sweep-dense-bytes", type=float, default=20e9,
+                    help="largest dense score matrix materialised for the recall check")
     args = ap.parse_args()
+    if args.sweep:
+        if args.workload == "long" and not args.sweep_values:
+            args.workload = "v4flash"
+        run_sweep(args)
+        return
     world, rank, local = dist_setup(args)
     args.gpus = world if world > 1 else args.gpus
     try:
