@@ -53,6 +53,10 @@ def test_workspace_bytes_host_arithmetic(lib):
     # pools fit in shared memory: header only
     assert si.workspace_bytes(1, 262144, 65536, 64, 128, 4, 512) == 256
     assert si.workspace_bytes(1, 2048, 512, 8, 64, 4, 64) == 256
+    # k = 1024 at H_I=64 still fits (1856-entry pools, spare room k + 768)
+    assert si.workspace_bytes(1, 65536, 16384, 64, 128, 4, 1024) == 256
+    # k = 600 at H_I=32 does not: 148 CTAs x 8 queries x 2400-entry (4k) pools x 8 bytes
+    assert si.workspace_bytes(1, 98304, 24576, 32, 128, 4, 600) == 256 + 148 * 8 * 2400 * 8
     # k = 2048 at H_I=64: 148 CTAs x 4 queries x 8192-entry (4k) pools x 8 bytes
     assert si.workspace_bytes(4, 131072, 32768, 64, 128, 4, 2048) == 256 + 148 * 4 * 8192 * 8
     # independent of S and T (never O(S*T))

@@ -141,13 +141,22 @@ def test_timeout_selftest_reports_and_context_survives():
 
 
 def test_workspace_pools_with_streamed_cuts():
-    """k=1024 at H_I=64 puts the candidate pools in the workspace (4k entries
-    per query), and rows long enough that the pools are cut while more than
-    2048 entries are held: the streamed (not register-held) cut path."""
-    wl = synth.Workload("ws_pools", 1, 98304, 4, 64, 128, 1024)
+    """k=600 at H_I=32 puts the candidate pools in the workspace (4k = 2400
+    entries per query), and rows long enough that the pools are cut while
+    more than 2048 entries are held: the streamed (not register-held) cut
+    path, with the shared-memory exact-cut buffer."""
+    wl = synth.Workload("ws_pools", 1, 98304, 4, 32, 128, 600)
     q, w, kc = synth.generate(wl, seed=21, device=DEV)
     b_rows, t_rows = gh.sampled_rows(wl.B, wl.S, wl.m, wl.k, n=256)
     gh.check_against_oracle(q, w, kc, wl.m, wl.k, b_rows, t_rows, where="ws pools")
+
+
+def test_shared_memory_pools_at_k1024():
+    """k=1024 at H_I=64: 1856-entry pools in shared memory, cut often."""
+    wl = synth.Workload("smem_k1024", 1, 65536, 4, 64, 128, 1024)
+    q, w, kc = synth.generate(wl, seed=23, device=DEV)
+    b_rows, t_rows = gh.sampled_rows(wl.B, wl.S, wl.m, wl.k, n=256)
+    gh.check_against_oracle(q, w, kc, wl.m, wl.k, b_rows, t_rows, where="smem k=1024")
 
 
 @pytest.mark.parametrize("name", ["v4flash", "long"])
