@@ -461,7 +461,7 @@ def main():
     ap.add_argument("--steps", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="long")
+    ap.add_argument("--workload", default=None, help="long (default), or v4flash for --sweep")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
@@ -475,9 +475,9 @@ def main():
     ap.add_argument("--sweep-dense-bytes", type=float, default=20e9,
                     help="largest dense score matrix materialised for the recall check")
     args = ap.parse_args()
+    if args.workload is None:
+        args.workload = "v4flash" if args.sweep else "long"
     if args.sweep:
-        if args.workload == "long" and not args.sweep_values:
-            args.workload = "v4flash"
         run_sweep(args)
         return
     world, rank, local = dist_setup(args)

@@ -726,36 +726,41 @@ __device__ __noinline__ uint64_t cut_pool(uint64_t* pq, PoolRegions rg, int k, u
 }
 
 // Writes the k best keys of one query's pool (or all, when fewer), unordered,
-// to its output row, then pads the row with (-1, -inf); by the half.
-__device__ __noinline__ void emit_best(const uint64_t* pq, PoolRegions rg, int k, CutScratch& cs, int tid,
+// to its output row, then pads the row with (-1, -inf); by the half.  The
+// kept keys are packed to the front of the pool first, so that the row is
+// written with coalesced stores.
+__device__ __noinline__ void emit_best(uint64_t* pq, PoolRegions rg, int k, CutScratch& cs, int tid,
                                        uint32_t bar_id, uint32_t& phase, int32_t* out_idx, float* out_score,
                                        uint64_t* big, int big_cap) {
-    auto emit = [&](uint64_t x, uint32_t pos) {
-        out_idx[pos] = key_index(x);
-        out_score[pos] = key_score(x);
-    };
+    auto pack = [&](uint64_t x, uint32_t pos) { pq[pos] = x; };
+    const uint32_t ku = static_cast<uint32_t>(k);
     uint32_t out;
     if (rg.total() <= 128 * kRegKeys) {
         RegKeys rk;
         rk.load(pq, rg, tid);
-        const uint32_t ku = static_cast<uint32_t>(k);
         const uint64_t L =
             rk.n <= k ? 0ull
             : big     ? half_select_bound<true>(rk, pq, rg, k, ku, cs, tid, bar_id, phase, big, big_cap)
                       : half_select_bound(rk, pq, rg, k, ku, cs, tid, bar_id, phase);
-        out = half_walk_reg(rk, L, cs, tid, bar_id, phase, emit);
+        out = half_walk_reg(rk, L, cs, tid, bar_id, phase, pack);
     } else {
         const StreamKeys sk{pq, rg};
-        const uint32_t ku = static_cast<uint32_t>(k);
         const uint64_t L =
             rg.total() <= k ? 0ull
             : big           ? half_select_bound<true>(sk, pq, rg, k, ku, cs, tid, bar_id, phase, big, big_cap)
                             : half_select_bound(sk, pq, rg, k, ku, cs, tid, bar_id, phase);
-        out = half_walk_kept(pq, rg, L, cs, tid, bar_id, phase, emit);
+        out = half_walk_kept(pq, rg, L, cs, tid, bar_id, phase, pack);
     }
-    for (int i = static_cast<int>(out) + tid; i < k; i += 128) {
-        out_idx[i] = -1;
-        out_score[i] = -__int_as_float(0x7f800000);
+    bar_sync(bar_id, 128);  // the packed keys are visible to the whole half
+    for (int i = tid; i < k; i += 128) {
+        if (i < static_cast<int>(out)) {
+            const uint64_t x = pq[i];
+            out_idx[i] = key_index(x);
+            out_score[i] = key_score(x);
+        } else {
+            out_idx[i] = -1;
+            out_score[i] = -__int_as_float(0x7f800000);
+        }
     }
 }
 
