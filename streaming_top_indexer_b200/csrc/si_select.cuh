@@ -509,6 +509,32 @@ __device__ __noinline__ uint64_t half_radix_bound(const uint64_t* pool, const Po
     return prefix;  // decided bits of the bucket, zeros below: its lowest key
 }
 
+// Warp 0 draws min(n, 32) keys at evenly spaced virtual positions and places
+// each at its rank among them (keys are distinct): cs.srt[0..ns) sorted
+// descending, 0 past the last.  Also clears cs.ncand.  Ends with a barrier of
+// the half; returns ns.
+__device__ __forceinline__ int half_samples(const uint64_t* pool, const PoolRegions& rg, CutScratch& cs, int tid,
+                                            uint32_t bar_id) {
+    const int lane = tid & 31;
+    const int n = rg.total();
+    const int ns = n < 32 ? n : 32;
+    if (tid < 32) {
+        const uint64_t me = lane < ns ? pool[region_addr(rg, n >= 32 ? (lane * n) >> 5 : lane)] : 0ull;
+        cs.cand[lane] = me;
+        __syncwarp();
+        int r = lane;
+        if (lane < ns) {
+            r = 0;
+#pragma unroll 8
+            for (int i = 0; i < 32; ++i) r += cs.cand[i] > me ? 1 : 0;
+        }
+        cs.srt[r] = me;
+    }
+    if (tid == 0) cs.ncand = 0;
+    bar_sync(bar_id, 128);
+    return ns;
+}
+
 // Lower bound L of the best keys in the regions, by the 128 threads of one
 // epilogue half: k <= #(keys >= L) <= max_keep (max_keep == k: exactly the k
 // best).  Needs n > k.
@@ -529,24 +555,8 @@ __device__ __forceinline__ uint64_t half_select_bound(const Keys& keys, const ui
                                                       int k, uint32_t max_keep, CutScratch& cs, int tid,
                                                       uint32_t bar_id, uint32_t& phase, uint64_t* big = nullptr,
                                                       int big_cap = 0) {
-    const int lane = tid & 31;
     const int n = rg.total();
-    const int ns = n < 32 ? n : 32;
-    if (tid < 32) {
-        // Samples are distinct keys; each is placed at its rank among them.
-        const uint64_t me = lane < ns ? pool[region_addr(rg, n >= 32 ? (lane * n) >> 5 : lane)] : 0ull;
-        cs.cand[lane] = me;
-        __syncwarp();
-        int r = lane;
-        if (lane < ns) {
-            r = 0;
-#pragma unroll 8
-            for (int i = 0; i < 32; ++i) r += cs.cand[i] > me ? 1 : 0;
-        }
-        cs.srt[r] = me;
-    }
-    if (tid == 0) cs.ncand = 0;
-    bar_sync(bar_id, 128);
+    const int ns = half_samples(pool, rg, cs, tid, bar_id);
     // c(r) = #(keys >= srt[r]) grows with r; c(-1) = 0 (no bound), c(ns) = n (bound 0)
     const uint32_t ku = static_cast<uint32_t>(k);
     const uint32_t target = max_keep > ku ? (ku + max_keep) / 2u : ku;
@@ -618,6 +628,67 @@ __device__ __forceinline__ uint64_t half_select_bound(const Keys& keys, const ui
     }
     bar_sync(bar_id, 128);
     return cs.xch[0];
+}
+
+// The exact k-th key of a large pool (workspace pools, which get a shared-
+// memory buffer `big`) in one pass over the keys: after the samples, the keys
+// above a window of samples around the predicted rank of the k-th key are
+// counted and the keys inside the window gathered into `big` (sized to fill
+// about half of it); when the k-th key falls inside, the sample select runs
+// on the gathered keys.  Returns false, with nothing decided, when it does
+// not or the window overflowed the buffer.  Needs n > k.
+template <typename Keys>
+__device__ __forceinline__ bool half_window_bound(const Keys& keys, const uint64_t* pool, const PoolRegions& rg, int k,
+                                                  CutScratch& cs, int tid, uint32_t bar_id, uint32_t& phase,
+                                                  uint64_t* big, int big_cap, uint64_t& L) {
+    const int n = rg.total();
+    const int ns = half_samples(pool, rg, cs, tid, bar_id);
+    const uint32_t ku = static_cast<uint32_t>(k);
+    // sample r has about (r + 1) * n / (ns + 1) keys at or above it
+    const int per_gap = n / (ns + 1) + 1;
+    int w = (big_cap / 2) / per_gap;  // sample gaps in the window
+    w = w < 2 ? 2 : w;
+    const int r0 = static_cast<int>((static_cast<long long>(ku) * (ns + 1) + n - 1) / n) - 1;
+    int a = r0 - w / 2;  // window [srt[b], srt[a]); a = -1: no upper end
+    a = a < -1 ? -1 : (a > ns - 1 ? ns - 1 : a);
+    const int b = a + w > ns ? ns : a + w;  // b = ns: no lower end
+    const uint64_t upper = a >= 0 ? cs.srt[a] : ~0ull;
+    const uint64_t lower = b < ns ? cs.srt[b] : 0ull;
+    const uint32_t cap = static_cast<uint32_t>(big_cap);
+    uint32_t above = 0;
+    keys.for_each(tid, [&](uint64_t x) {
+        if (x >= upper) {
+            ++above;
+        } else if (x >= lower) {
+            const uint32_t slot = atomicAdd(&cs.ncand, 1u);
+            if (slot < cap) big[slot] = x;
+        }
+    });
+    above = half_sum(above, cs, tid, bar_id, phase);  // its barrier also completes the gather
+    const uint32_t m = cs.ncand;
+    if (m > cap || above >= ku || above + m < ku) return false;  // uniform over the half
+    const uint32_t kb = ku - above;  // the k-th key is the kb-th of the window
+    if (kb == m) {
+        L = lower;  // the window's smallest key (b < ns here, since n > k)
+        return true;
+    }
+    PoolRegions one;
+    one.start[0] = 0;
+    one.len[0] = static_cast<int>(m);
+#pragma unroll
+    for (int r2 = 1; r2 < 5; ++r2) {
+        one.start[r2] = static_cast<int>(m);
+        one.len[r2] = 0;
+    }
+    if (m <= 128u * kRegKeys) {
+        RegKeys rk;
+        rk.load(big, one, tid);
+        L = half_select_bound(rk, big, one, static_cast<int>(kb), kb, cs, tid, bar_id, phase);
+    } else {
+        const StreamKeys sk{big, one};
+        L = half_select_bound(sk, big, one, static_cast<int>(kb), kb, cs, tid, bar_id, phase);
+    }
+    return true;
 }
 
 // Hands every region entry >= L, with a distinct output position in
@@ -717,9 +788,11 @@ __device__ __noinline__ uint64_t cut_pool(uint64_t* pq, PoolRegions rg, int k, u
         kept = half_walk_reg(rk, L, cs, tid, bar_id, phase, [&](uint64_t x, uint32_t pos) { pq[pos] = x; });
     } else {
         const StreamKeys sk{pq, rg};
-        if (rg.total() > k)
-            L = big ? half_select_bound<true>(sk, pq, rg, k, max_keep, cs, tid, bar_id, phase, big, big_cap)
-                    : half_select_bound(sk, pq, rg, k, max_keep, cs, tid, bar_id, phase);
+        if (rg.total() > k) {
+            if (!(big && half_window_bound(sk, pq, rg, k, cs, tid, bar_id, phase, big, big_cap, L)))
+                L = big ? half_select_bound<true>(sk, pq, rg, k, max_keep, cs, tid, bar_id, phase, big, big_cap)
+                        : half_select_bound(sk, pq, rg, k, max_keep, cs, tid, bar_id, phase);
+        }
         kept = half_walk_kept(pq, rg, L, cs, tid, bar_id, phase, [&](uint64_t x, uint32_t pos) { pq[pos] = x; });
     }
     return L;
@@ -745,10 +818,12 @@ __device__ __noinline__ void emit_best(uint64_t* pq, PoolRegions rg, int k, CutS
         out = half_walk_reg(rk, L, cs, tid, bar_id, phase, pack);
     } else {
         const StreamKeys sk{pq, rg};
-        const uint64_t L =
-            rg.total() <= k ? 0ull
-            : big           ? half_select_bound<true>(sk, pq, rg, k, ku, cs, tid, bar_id, phase, big, big_cap)
-                            : half_select_bound(sk, pq, rg, k, ku, cs, tid, bar_id, phase);
+        uint64_t L = 0ull;
+        if (rg.total() > k) {
+            if (!(big && half_window_bound(sk, pq, rg, k, cs, tid, bar_id, phase, big, big_cap, L)))
+                L = big ? half_select_bound<true>(sk, pq, rg, k, ku, cs, tid, bar_id, phase, big, big_cap)
+                        : half_select_bound(sk, pq, rg, k, ku, cs, tid, bar_id, phase);
+        }
         out = half_walk_kept(pq, rg, L, cs, tid, bar_id, phase, pack);
     }
     bar_sync(bar_id, 128);  // the packed keys are visible to the whole half

@@ -87,11 +87,26 @@ __global__ void __launch_bounds__(K2 / 8) sort_rows_block_kernel(int32_t* __rest
     if (row >= rows) return;
     int32_t* ri = idx + row * k;
     float* rs = score + row * k;
+    // A thread's eight entries are 32 contiguous bytes of each array: two
+    // 16-byte accesses when the row is 16-byte aligned and complete.
+    const bool vec = ((reinterpret_cast<uintptr_t>(ri) | reinterpret_cast<uintptr_t>(rs)) & 15u) == 0 &&
+                     tid * E + E <= k;
     uint64_t v[E];
+    if (vec) {
+        const int4 i0 = reinterpret_cast<const int4*>(ri + tid * E)[0];
+        const int4 i1 = reinterpret_cast<const int4*>(ri + tid * E)[1];
+        const float4 s0 = reinterpret_cast<const float4*>(rs + tid * E)[0];
+        const float4 s1 = reinterpret_cast<const float4*>(rs + tid * E)[1];
+        const int iv[E] = {i0.x, i0.y, i0.z, i0.w, i1.x, i1.y, i1.z, i1.w};
+        const float sv[E] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
 #pragma unroll
-    for (int e = 0; e < E; ++e) {
-        const int i = tid * E + e;
-        v[e] = (i < k) ? pack_key(rs[i], static_cast<uint32_t>(ri[i])) : 0ull;
+        for (int e = 0; e < E; ++e) v[e] = pack_key(sv[e], static_cast<uint32_t>(iv[e]));
+    } else {
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+            const int i = tid * E + e;
+            v[e] = (i < k) ? pack_key(rs[i], static_cast<uint32_t>(ri[i])) : 0ull;
+        }
     }
     int buf = 0;
 #pragma unroll
@@ -134,12 +149,23 @@ __global__ void __launch_bounds__(K2 / 8) sort_rows_block_kernel(int32_t* __rest
             }
         }
     }
+    if (vec) {
+        reinterpret_cast<int4*>(ri + tid * E)[0] =
+            make_int4(key_index(v[0]), key_index(v[1]), key_index(v[2]), key_index(v[3]));
+        reinterpret_cast<int4*>(ri + tid * E)[1] =
+            make_int4(key_index(v[4]), key_index(v[5]), key_index(v[6]), key_index(v[7]));
+        reinterpret_cast<float4*>(rs + tid * E)[0] =
+            make_float4(key_score(v[0]), key_score(v[1]), key_score(v[2]), key_score(v[3]));
+        reinterpret_cast<float4*>(rs + tid * E)[1] =
+            make_float4(key_score(v[4]), key_score(v[5]), key_score(v[6]), key_score(v[7]));
+    } else {
 #pragma unroll
-    for (int e = 0; e < E; ++e) {
-        const int i = tid * E + e;
-        if (i < k) {
-            ri[i] = key_index(v[e]);
-            rs[i] = key_score(v[e]);
+        for (int e = 0; e < E; ++e) {
+            const int i = tid * E + e;
+            if (i < k) {
+                ri[i] = key_index(v[e]);
+                rs[i] = key_score(v[e]);
+            }
         }
     }
 }
