@@ -75,6 +75,29 @@ SI_API si_status si_indexer_topk(const void* q, const float* w, const void* kc,
                           int32_t* out_idx, float* out_score,
                           void* workspace, size_t workspace_bytes, si_stream_t stream);
 
+/* si_indexer_topk for the query rows [t_begin, t_end) of every batch only.
+ * The method selects each query row's keys on its own (StreamIndex:
+ * Memory-Bounded Compressed Sparse Attention via Streaming Top-k, Abstract),
+ * so rows can be computed in windows.  This lets a caller overlap the
+ * host-to-device copy of later rows, and the copy back of earlier results,
+ * with the computation of a window.
+ *   q, w, out_idx, out_score: the WHOLE [B,S,...] tensors (same layout and
+ *     alignment rules as si_indexer_topk); only the window's rows of q and w
+ *     are read and only the window's rows of the outputs are written.
+ *   kc: the whole [B,T,d_I] tensor (keys are visible by the absolute row t).
+ *   t_begin: a multiple of 256; t_end: a multiple of 256, or S;
+ *     0 <= t_begin <= t_end <= S (else SI_ERR_INVALID_ARG, nothing enqueued).
+ *   workspace: as si_indexer_topk.  Its header (device error word) is reset
+ *     only by a call with t_begin == 0, so after a sequence of windows that
+ *     starts at row 0, si_check_device_status reports a failure of any of
+ *     them.  Windows enqueued on different streams with one workspace race.
+ * Result rows are identical to those of si_indexer_topk. */
+SI_API si_status si_indexer_topk_rows(const void* q, const float* w, const void* kc,
+                               int64_t B, int64_t S, int64_t T, int H_I, int d_I, int m, int k,
+                               int64_t t_begin, int64_t t_end,
+                               int32_t* out_idx, float* out_score,
+                               void* workspace, size_t workspace_bytes, si_stream_t stream);
+
 /* First stage of si_indexer_topk alone: the fused scoring + selection kernel.
  * Leaves each row's top-k set in out_idx/out_score unordered (padding at the
  * tail).  Does not reset the workspace header.  Exposed so that the stages

@@ -53,6 +53,8 @@ def _declare(lib):
         fn = getattr(lib, name)
         fn.restype = c.c_int
         fn.argtypes = topk_args
+    lib.si_indexer_topk_rows.restype = c.c_int
+    lib.si_indexer_topk_rows.argtypes = topk_args[:10] + [i64, i64] + topk_args[10:]
     lib.si_sort_topk.restype = c.c_int
     lib.si_sort_topk.argtypes = [vp, vp, i64, i32, vp]
     lib.si_indexer_scores.restype = c.c_int
@@ -168,6 +170,21 @@ def indexer_topk(q, w, kc, m: int, k: int, out_idx=None, out_score=None, workspa
     return _topk_call("si_indexer_topk", q, w, kc, m, k, out_idx, out_score, workspace, stream)
 
 
+def indexer_topk_rows(q, w, kc, m: int, k: int, t_begin: int, t_end: int, out_idx, out_score, workspace,
+                      stream=None):
+    """Query rows [t_begin, t_end) of every batch (si_indexer_topk_rows): the
+    whole q, w and output tensors are passed, only the window's rows are read
+    and written.  t_begin is a multiple of 256, t_end a multiple of 256 or S."""
+    B, S, T, H, D = _dims(q, w, kc)
+    _need(out_idx, "out_idx", torch.int32, 3)
+    _need(out_score, "out_score", torch.float32, 3)
+    _check(load_library().si_indexer_topk_rows(q.data_ptr(), w.data_ptr(), kc.data_ptr() if T > 0 else None, B, S,
+                                               T, H, D, m, k, int(t_begin), int(t_end), out_idx.data_ptr(),
+                                               out_score.data_ptr(), workspace.data_ptr(), workspace.numel(),
+                                               _stream(stream)), "si_indexer_topk_rows")
+    return out_idx, out_score
+
+
 def select_topk(q, w, kc, m: int, k: int, out_idx=None, out_score=None, workspace=None, stream=None):
     """First stage only (si_select_topk): each row's top-k set, unordered."""
     return _topk_call("si_select_topk", q, w, kc, m, k, out_idx, out_score, workspace, stream)
@@ -211,14 +228,28 @@ def selftest_timeout(workspace, limit_ns: int, stream=None) -> int:
     return check_device_status(workspace, stream)
 
 
-def indexer_topk_host(q, w, kc, m: int, k: int, device="cuda", buffers=None, stream=None):
-    """End-to-end call on host tensors: copies q, w, kc to the GPU, runs
-    si_indexer_topk and copies (idx, score) back into host tensors.
+def host_row_windows(S: int, chunks: int):
+    """Row windows of the pipelined host path: boundaries on multiples of 256
+    (the last window ends at S), about S/chunks rows each, no empty window."""
+    step = max(256, -(-S // max(1, chunks)) // 256 * 256)
+    bounds = list(range(0, S, step)) + [S]
+    return [(bounds[i], bounds[i + 1]) for i in range(len(bounds) - 1)]
+
+
+def indexer_topk_host(q, w, kc, m: int, k: int, device="cuda", buffers=None, stream=None, chunks: int = 8):
+    """End-to-end call on host tensors: copies q, w, kc to the GPU, runs the
+    indexer and copies (idx, score) back into host tensors.
+
+    The rows are processed in windows (si_indexer_topk_rows): while window c
+    runs, the inputs of window c+1 are copied in and the results of window
+    c-1 are copied out, on two copy streams.  Host tensors should be pinned
+    for the copies to overlap.
 
     ``buffers`` may hold preallocated device tensors ("q","w","kc","idx",
-    "score","ws") and pinned host outputs ("idx_h","score_h") to reuse.
-    Returns (idx_h, score_h); the copies are asynchronous on ``stream`` and
-    complete when the stream is synchronised.
+    "score","ws"), pinned host outputs ("idx_h","score_h") and the copy
+    streams to reuse.  Returns (idx_h, score_h); everything is asynchronous
+    and complete once ``stream`` (default: torch's current stream) is
+    synchronised.
     """
     b = {} if buffers is None else buffers
     dev = torch.device(device)
@@ -233,12 +264,34 @@ def indexer_topk_host(q, w, kc, m: int, k: int, device="cuda", buffers=None, str
         b["ws"] = torch.empty(workspace_bytes(B, S, T, H, D, m, k), dtype=torch.uint8, device=dev)
         b["idx_h"] = torch.empty((B, S, k), dtype=torch.int32, pin_memory=True)
         b["score_h"] = torch.empty((B, S, k), dtype=torch.float32, pin_memory=True)
+        b["s_in"] = torch.cuda.Stream(dev)
+        b["s_out"] = torch.cuda.Stream(dev)
     s = stream if stream is not None else torch.cuda.current_stream(dev)
-    with torch.cuda.stream(s):
-        b["q"].copy_(q, non_blocking=True)
-        b["w"].copy_(w, non_blocking=True)
+    s_in, s_out = b["s_in"], b["s_out"]
+    windows = host_row_windows(S, chunks) if S > 0 else []
+    # The copy-in stream starts after everything already queued on `stream`
+    # (which includes the previous call's copy-out).
+    s_in.wait_stream(s)
+    with torch.cuda.stream(s_in):
         b["kc"].copy_(kc, non_blocking=True)
-        indexer_topk(b["q"], b["w"], b["kc"], m, k, b["idx"], b["score"], b["ws"], s)
-        b["idx_h"].copy_(b["idx"], non_blocking=True)
-        b["score_h"].copy_(b["score"], non_blocking=True)
+        in_done = []
+        for t0, t1 in windows:
+            b["q"][:, t0:t1].copy_(q[:, t0:t1], non_blocking=True)
+            b["w"][:, t0:t1].copy_(w[:, t0:t1], non_blocking=True)
+            ev = torch.cuda.Event()
+            ev.record(s_in)
+            in_done.append(ev)
+    out_ready = []
+    for (t0, t1), ev in zip(windows, in_done):
+        s.wait_event(ev)
+        indexer_topk_rows(b["q"], b["w"], b["kc"], m, k, t0, t1, b["idx"], b["score"], b["ws"], s)
+        done = torch.cuda.Event()
+        done.record(s)
+        out_ready.append(done)
+    with torch.cuda.stream(s_out):
+        for (t0, t1), ev in zip(windows, out_ready):
+            s_out.wait_event(ev)
+            b["idx_h"][:, t0:t1].copy_(b["idx"][:, t0:t1], non_blocking=True)
+            b["score_h"][:, t0:t1].copy_(b["score"][:, t0:t1], non_blocking=True)
+    s.wait_stream(s_out)
     return b["idx_h"], b["score_h"]

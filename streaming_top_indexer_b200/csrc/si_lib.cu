@@ -30,6 +30,9 @@ si_status cuda_fail(const char* where, cudaError_t e) {
 
 constexpr int kMaxCtas = 148;                 // persistent CTAs (one per B200 SM)
 constexpr size_t kHeaderBytes = 256;          // error word + reserved
+// Row windows of si_indexer_topk_rows start (and, except at S, end) on
+// multiples of this, a multiple of every unit's query count (256/H_I).
+constexpr int64_t kRowAlign = 256;
 constexpr uint32_t kMaxDynSmem = 232448;      // 227 KB opt-in per block on sm_100
 constexpr uint32_t kMinDynSmem = 120 * 1024;  // > half an SM: one CTA per SM, so
                                               // two CTAs never compete for TMEM
@@ -158,7 +161,8 @@ int device_sms(int dev) {
 
 template <int H, int D>
 si_status launch_select_t(const void* q, const float* w, const void* kc, int64_t B, int64_t S, int64_t T, int m,
-                          int k, int32_t* out_idx, float* out_score, float* dense, void* ws, cudaStream_t stream) {
+                          int k, int32_t* out_idx, float* out_score, float* dense, void* ws, cudaStream_t stream,
+                          int64_t t_lo, int64_t t_hi) {
     using C = si::SelCfg<H, D>;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return SI_ERR_CUDA;
@@ -173,7 +177,9 @@ si_status launch_select_t(const void* q, const float* w, const void* kc, int64_t
     p.k = dense ? 1 : k;
     const PoolPlan pp = dense ? PoolPlan{true, 0} : pool_plan(H, D, p.k);
     p.P = pp.P;
-    p.nblk = (S + C::QT - 1) / C::QT;
+    p.t_lo = t_lo;
+    p.t_hi = t_hi;
+    p.nblk = (t_hi - t_lo + C::QT - 1) / C::QT;
     p.units = B * p.nblk;
     p.out_idx = out_idx;
     p.out_score = out_score;
@@ -218,12 +224,14 @@ si_status launch_select_t(const void* q, const float* w, const void* kc, int64_t
     return e == cudaSuccess ? SI_OK : cuda_fail("select kernel launch", e);
 }
 
+// Query rows [t_lo, t_hi) of every batch; the whole problem is [0, S).
 si_status launch_select(const void* q, const float* w, const void* kc, int64_t B, int64_t S, int64_t T, int H, int D,
                         int m, int k, int32_t* out_idx, float* out_score, float* dense, void* ws,
-                        cudaStream_t stream) {
+                        cudaStream_t stream, int64_t t_lo = 0, int64_t t_hi = -1) {
+    if (t_hi < 0) t_hi = S;
 #define SI_CASE(HH, DD)     \
     if (H == HH && D == DD) \
-        return launch_select_t<HH, DD>(q, w, kc, B, S, T, m, k, out_idx, out_score, dense, ws, stream);
+        return launch_select_t<HH, DD>(q, w, kc, B, S, T, m, k, out_idx, out_score, dense, ws, stream, t_lo, t_hi);
     SI_CASE(8, 64) SI_CASE(8, 128) SI_CASE(16, 64) SI_CASE(16, 128)
     SI_CASE(32, 64) SI_CASE(32, 128) SI_CASE(64, 64) SI_CASE(64, 128)
 #undef SI_CASE
@@ -296,6 +304,35 @@ si_status si_indexer_topk(const void* q, const float* w, const void* kc, int64_t
     st = launch_select(q, w, kc, B, S, T, H_I, d_I, m, k, out_idx, out_score, nullptr, workspace, s);
     if (st != SI_OK) return st;
     return si_sort_topk(out_idx, out_score, B * S, k, stream);
+}
+
+si_status si_indexer_topk_rows(const void* q, const float* w, const void* kc, int64_t B, int64_t S, int64_t T,
+                               int H_I, int d_I, int m, int k, int64_t t_begin, int64_t t_end, int32_t* out_idx,
+                               float* out_score, void* workspace, size_t workspace_bytes, si_stream_t stream) {
+    si_status st = check_topk(q, w, kc, B, S, T, H_I, d_I, m, k, out_idx, out_score, workspace, workspace_bytes);
+    if (st != SI_OK) return st;
+    if (t_begin < 0 || t_end > S || t_begin > t_end) return SI_ERR_INVALID_ARG;
+    if (t_begin % kRowAlign != 0 || (t_end % kRowAlign != 0 && t_end != S)) return SI_ERR_INVALID_ARG;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (t_begin == 0 && cudaMemsetAsync(workspace, 0, kHeaderBytes, s) != cudaSuccess) return SI_ERR_CUDA;
+    if (t_begin == t_end) return SI_OK;
+    const int64_t n = t_end - t_begin;
+    if (T == 0) {
+        for (int64_t b = 0; b < B; ++b) {
+            const int64_t off = (b * S + t_begin) * k;
+            st = launch_pad(out_idx + off, out_score + off, n * k, s);
+            if (st != SI_OK) return st;
+        }
+        return SI_OK;
+    }
+    st = launch_select(q, w, kc, B, S, T, H_I, d_I, m, k, out_idx, out_score, nullptr, workspace, s, t_begin, t_end);
+    if (st != SI_OK) return st;
+    for (int64_t b = 0; b < B; ++b) {
+        const int64_t off = (b * S + t_begin) * k;
+        st = si_sort_topk(out_idx + off, out_score + off, n, k, stream);
+        if (st != SI_OK) return st;
+    }
+    return SI_OK;
 }
 
 si_status si_indexer_scores(const void* q, const float* w, const void* kc, int64_t B, int64_t S, int64_t T, int H_I,

@@ -75,7 +75,8 @@ struct SelectParams {
     int64_t B, S, T;
     int m, k;
     int P;              // pool capacity per query (multiple of 32, >= k + 288)
-    int64_t nblk;       // query blocks per batch
+    int64_t t_lo, t_hi; // query rows [t_lo, t_hi) of every batch are computed
+    int64_t nblk;       // query blocks per batch in [t_lo, t_hi)
     int64_t units;      // B * nblk
     int32_t* out_idx;   // [B,S,k]
     float* out_score;   // [B,S,k]
@@ -170,13 +171,14 @@ struct UnitInfo {
     int ntiles;
 };
 
-// Units are ordered longest first: unit u is query block nblk-1-u/B of batch u%B.
+// Units are ordered longest first: unit u is query block nblk-1-u/B (of the
+// rows [t_lo, t_hi)) of batch u%B.
 __device__ __forceinline__ UnitInfo decode_unit(int64_t u, const SelectParams& p, int QT) {
     UnitInfo ui;
     const int64_t blk = p.nblk - 1 - u / p.B;
     ui.b = u % p.B;
-    ui.t0 = blk * QT;
-    const int64_t tend = (ui.t0 + QT < p.S) ? ui.t0 + QT : p.S;
+    ui.t0 = p.t_lo + blk * QT;
+    const int64_t tend = (ui.t0 + QT < p.t_hi) ? ui.t0 + QT : p.t_hi;
     int64_t vmax = tend / p.m;  // keys visible to query tend-1
     if (vmax > p.T) vmax = p.T;
     ui.ntiles = static_cast<int>((vmax + 127) / 128);
@@ -1067,7 +1069,7 @@ __global__ void __launch_bounds__(SelCfg<H, D>::THREADS, 1)
                 kp[q] = 0u;
                 cw[q] = 0u;
                 const int64_t t = ui.t0 + half * C::QH + q;
-                int64_t v = (t < p.S) ? (t + 1) / p.m : 0;
+                int64_t v = (t < p.t_hi) ? (t + 1) / p.m : 0;
                 vis[q] = static_cast<int32_t>(v < p.T ? v : p.T);
             }
             const bool tr_lead = true;
@@ -1211,7 +1213,7 @@ __global__ void __launch_bounds__(SelCfg<H, D>::THREADS, 1)
                 for (int q = 0; q < C::QH; ++q) {
                     const int qi = half * C::QH + q;
                     const int64_t t = ui.t0 + qi;
-                    if (t >= p.S) continue;  // uniform over the half
+                    if (t >= p.t_hi) continue;  // uniform over the half
                     const int64_t row = (ui.b * p.S + t) * static_cast<int64_t>(k);
                     emit_best(pool + qi * P, pool_regions(kp[q], fw(q), cntw[half][q]), k, cs, htid, bar_id, cphase,
                               p.out_idx + row, p.out_score + row, big, C::STREAM_CAND);

@@ -97,3 +97,31 @@ def test_python_binding_refuses_cpu_tensors():
     kc = torch.zeros((1, 2, 128), dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         si.indexer_topk(q, w, kc, 4, 4)
+
+
+def call_rows(lib, t0, t1, S=1000, **kw):
+    a = dict(q=16, w=16, kc=16, B=1, T=250, H=64, D=128, m=4, k=4, oi=16, os_=16, ws=16, wsb=1 << 20)
+    a.update(kw)
+    return lib.si_indexer_topk_rows(a["q"], a["w"], a["kc"], a["B"], S, a["T"], a["H"], a["D"], a["m"], a["k"],
+                                    t0, t1, a["oi"], a["os_"], a["ws"], a["wsb"], None)
+
+
+def test_row_window_arguments_before_any_cuda_call(lib):
+    assert call_rows(lib, 100, 512) == 1     # window start not a multiple of 256
+    assert call_rows(lib, 0, 300) == 1       # window end neither a multiple of 256 nor S
+    assert call_rows(lib, 512, 256) == 1     # start after end
+    assert call_rows(lib, -256, 256) == 1
+    assert call_rows(lib, 0, 1024) == 1      # end past S
+    assert call_rows(lib, 0, 256, q=0) == 1  # the whole-problem checks still apply
+    assert call_rows(lib, 0, 256, H=12) == 2
+
+
+def test_host_row_windows():
+    for S, chunks in [(262144, 8), (65536, 8), (2048, 8), (300, 8), (100, 4), (257, 1), (4096, 3)]:
+        win = si.host_row_windows(S, chunks)
+        assert win[0][0] == 0 and win[-1][1] == S
+        for (a, b), (c, _) in zip(win, win[1:]):
+            assert b == c
+        for a, b in win:
+            assert a < b and a % 256 == 0 and (b % 256 == 0 or b == S)
+        assert len(win) <= max(1, chunks) + 1

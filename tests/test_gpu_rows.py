@@ -1,0 +1,70 @@
+"""Row windows (si_indexer_topk_rows) and the pipelined host path built on
+them: the same rows as the whole-problem call, bit for bit."""
+import pytest
+import torch
+
+import streaming_top_indexer_b200 as si
+from streaming_top_indexer_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+SHAPES = [
+    # B, S, T, H, D, m, k
+    (1, 1000, 250, 64, 128, 4, 64),
+    (2, 777, 300, 32, 128, 2, 100),
+    (1, 2000, 500, 64, 64, 4, 600),   # k > T
+    (3, 600, 40, 8, 128, 7, 5),       # T > S/m
+    (1, 1500, 375, 64, 128, 4, 2048),  # workspace pools
+]
+
+
+def inputs(B, S, T, H, D, m, k, seed):
+    wl = synth.Workload("rows", B, S, m, H, D, k)
+    return synth.generate(wl, seed=seed, device=DEV, T=T)
+
+
+@pytest.mark.parametrize("B,S,T,H,D,m,k", SHAPES)
+def test_windows_equal_whole_call(B, S, T, H, D, m, k):
+    q, w, kc = inputs(B, S, T, H, D, m, k, seed=S + 7)
+    ws = torch.zeros(si.workspace_bytes(B, S, T, H, D, m, k), dtype=torch.uint8, device=DEV)
+    ref_idx, ref_sc = si.indexer_topk(q, w, kc, m, k, workspace=ws)
+    assert si.check_device_status(ws) == 0
+    idx = torch.full((B, S, k), -7, dtype=torch.int32, device=DEV)
+    sc = torch.full((B, S, k), 7.0, dtype=torch.float32, device=DEV)
+    for t0, t1 in si.host_row_windows(S, 3):
+        si.indexer_topk_rows(q, w, kc, m, k, t0, t1, idx, sc, ws)
+    assert si.check_device_status(ws) == 0
+    assert torch.equal(idx, ref_idx)
+    assert torch.equal(sc.view(torch.int32), ref_sc.view(torch.int32))
+
+
+def test_window_touches_only_its_rows():
+    B, S, T, H, D, m, k = 2, 1024, 256, 64, 128, 4, 32
+    q, w, kc = inputs(B, S, T, H, D, m, k, seed=3)
+    ws = torch.zeros(si.workspace_bytes(B, S, T, H, D, m, k), dtype=torch.uint8, device=DEV)
+    ref_idx, ref_sc = si.indexer_topk(q, w, kc, m, k, workspace=ws)
+    idx = torch.full((B, S, k), -7, dtype=torch.int32, device=DEV)
+    sc = torch.full((B, S, k), 7.0, dtype=torch.float32, device=DEV)
+    si.indexer_topk_rows(q, w, kc, m, k, 256, 768, idx, sc, ws)
+    assert si.check_device_status(ws) == 0
+    assert torch.equal(idx[:, 256:768], ref_idx[:, 256:768])
+    assert torch.equal(sc[:, 256:768], ref_sc[:, 256:768])
+    assert torch.all(idx[:, :256] == -7) and torch.all(idx[:, 768:] == -7)
+    assert torch.all(sc[:, :256] == 7.0) and torch.all(sc[:, 768:] == 7.0)
+
+
+@pytest.mark.parametrize("chunks", [1, 4])
+def test_pipelined_host_path_equals_device_call(chunks):
+    B, S, T, H, D, m, k = 1, 4096, 1024, 64, 128, 4, 512
+    q, w, kc = inputs(B, S, T, H, D, m, k, seed=11)
+    ref_idx, ref_sc = si.indexer_topk(q, w, kc, m, k)
+    qh, wh, kch = q.cpu().pin_memory(), w.cpu().pin_memory(), kc.cpu().pin_memory()
+    bufs = {}
+    for _ in range(2):  # buffers and streams reused on the second call
+        idx_h, sc_h = si.indexer_topk_host(qh, wh, kch, m, k, device=DEV, buffers=bufs, chunks=chunks)
+        torch.cuda.current_stream().synchronize()
+        assert si.check_device_status(bufs["ws"]) == 0
+        assert torch.equal(idx_h, ref_idx.cpu())
+        assert torch.equal(sc_h.view(torch.int32), ref_sc.cpu().view(torch.int32))
