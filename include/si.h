@@ -87,10 +87,11 @@ SI_API si_status si_indexer_topk(const void* q, const float* w, const void* kc,
  *   kc: the whole [B,T,d_I] tensor (keys are visible by the absolute row t).
  *   t_begin: a multiple of 256; t_end: a multiple of 256, or S;
  *     0 <= t_begin <= t_end <= S (else SI_ERR_INVALID_ARG, nothing enqueued).
- *   workspace: as si_indexer_topk.  Its header (device error word) is reset
- *     only by a call with t_begin == 0, so after a sequence of windows that
- *     starts at row 0, si_check_device_status reports a failure of any of
- *     them.  Windows enqueued on different streams with one workspace race.
+ *   workspace: as si_indexer_topk.  Its header (device error word) is NOT
+ *     reset: reset it once with si_reset_device_status before a sequence of
+ *     windows, and si_check_device_status afterwards reports a failure of
+ *     any of them.  Windows enqueued on different streams with one
+ *     workspace race.
  * Result rows are identical to those of si_indexer_topk. */
 SI_API si_status si_indexer_topk_rows(const void* q, const float* w, const void* kc,
                                int64_t B, int64_t S, int64_t T, int H_I, int d_I, int m, int k,
@@ -121,6 +122,13 @@ SI_API si_status si_indexer_scores(const void* q, const float* w, const void* kc
                             int64_t B, int64_t S, int64_t T, int H_I, int d_I, int m,
                             float* out_scores, void* workspace, size_t workspace_bytes,
                             si_stream_t stream);
+
+/* Clears the device error word in the workspace header (a 256-byte
+ * asynchronous memset on `stream`), as si_indexer_topk does at its start.
+ * SI_ERR_INVALID_ARG for a null workspace, SI_ERR_MISALIGNED unless it is
+ * 16-byte aligned, SI_ERR_CUDA if the memset cannot be enqueued.  The paper
+ * has no counterpart; it serves sequences of si_indexer_topk_rows calls. */
+SI_API si_status si_reset_device_status(void* workspace, si_stream_t stream);
 
 /* Synchronises `stream`, then returns SI_OK or the device error recorded in
  * the workspace header by the last call that used it (SI_ERR_TIMEOUT), or

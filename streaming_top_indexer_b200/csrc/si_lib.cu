@@ -314,7 +314,6 @@ si_status si_indexer_topk_rows(const void* q, const float* w, const void* kc, in
     if (t_begin < 0 || t_end > S || t_begin > t_end) return SI_ERR_INVALID_ARG;
     if (t_begin % kRowAlign != 0 || (t_end % kRowAlign != 0 && t_end != S)) return SI_ERR_INVALID_ARG;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    if (t_begin == 0 && cudaMemsetAsync(workspace, 0, kHeaderBytes, s) != cudaSuccess) return SI_ERR_CUDA;
     if (t_begin == t_end) return SI_OK;
     const int64_t n = t_end - t_begin;
     if (T == 0) {
@@ -348,6 +347,13 @@ si_status si_indexer_scores(const void* q, const float* w, const void* kc, int64
     if (cudaMemsetAsync(workspace, 0, kHeaderBytes, s) != cudaSuccess) return SI_ERR_CUDA;
     if (T == 0) return SI_OK;
     return launch_select(q, w, kc, B, S, T, H_I, d_I, m, 1, nullptr, nullptr, out_scores, workspace, s);
+}
+
+si_status si_reset_device_status(void* workspace, si_stream_t stream) {
+    if (!workspace) return SI_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(workspace) & 15u) return SI_ERR_MISALIGNED;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    return cudaMemsetAsync(workspace, 0, kHeaderBytes, s) == cudaSuccess ? SI_OK : SI_ERR_CUDA;
 }
 
 si_status si_check_device_status(const void* workspace, si_stream_t stream) {

@@ -88,6 +88,8 @@ def test_argument_errors_before_any_cuda_call(lib):
     assert lib.si_sort_topk(0, 16, 4, 8, None) == 1
     assert lib.si_indexer_scores(16, 16, 16, 1, 8, 2, 64, 128, 4, 16, 16, 8, None) == 4
     assert lib.si_selftest_timeout(0, 256, 1000, None) == 1
+    assert lib.si_reset_device_status(0, None) == 1
+    assert lib.si_reset_device_status(24, None) == 3
 
 
 def test_python_binding_refuses_cpu_tensors():

@@ -33,7 +33,8 @@ def test_windows_equal_whole_call(B, S, T, H, D, m, k):
     assert si.check_device_status(ws) == 0
     idx = torch.full((B, S, k), -7, dtype=torch.int32, device=DEV)
     sc = torch.full((B, S, k), 7.0, dtype=torch.float32, device=DEV)
-    for t0, t1 in si.host_row_windows(S, 3):
+    si.reset_device_status(ws)
+    for t0, t1 in si.host_row_windows(S, 3)[::-1]:  # any order
         si.indexer_topk_rows(q, w, kc, m, k, t0, t1, idx, sc, ws)
     assert si.check_device_status(ws) == 0
     assert torch.equal(idx, ref_idx)
