@@ -129,6 +129,7 @@ struct SelCfg {
     // With the pools in the workspace, each epilogue group gets a buffer of
     // STREAM_CAND keys in shared memory for the exact cut of its large pools.
     static constexpr int STREAM_CAND = 3072;
+    static_assert(STREAM_CAND >= 2048, "final selections (k <= 2048) of workspace pools are packed into it");
     static constexpr uint32_t dyn_bytes(bool pool_in_smem, int P) {
         return OFF_POOL +
                (pool_in_smem ? static_cast<uint32_t>(QT) * P * 8u : static_cast<uint32_t>(NGROUPS * STREAM_CAND) * 8u) +
@@ -781,13 +782,14 @@ __device__ __noinline__ uint64_t cut_pool(uint64_t* pq, PoolRegions rg, int k, u
                                           CutScratch& cs, int tid, uint32_t bar_id, uint32_t& phase,
                                           uint32_t& kept, uint64_t* big, int big_cap) {
     uint64_t L = lb;
+    auto pack = [&](uint64_t x, uint32_t pos) { pq[pos] = x; };
     if (rg.total() <= 128 * kRegKeys) {
         RegKeys rk;
         rk.load(pq, rg, tid);
         if (rk.n > k)
             L = big ? half_select_bound<true>(rk, pq, rg, k, max_keep, cs, tid, bar_id, phase, big, big_cap)
                     : half_select_bound(rk, pq, rg, k, max_keep, cs, tid, bar_id, phase);
-        kept = half_walk_reg(rk, L, cs, tid, bar_id, phase, [&](uint64_t x, uint32_t pos) { pq[pos] = x; });
+        kept = half_walk_reg(rk, L, cs, tid, bar_id, phase, pack);
     } else {
         const StreamKeys sk{pq, rg};
         if (rg.total() > k) {
@@ -795,19 +797,21 @@ __device__ __noinline__ uint64_t cut_pool(uint64_t* pq, PoolRegions rg, int k, u
                 L = big ? half_select_bound<true>(sk, pq, rg, k, max_keep, cs, tid, bar_id, phase, big, big_cap)
                         : half_select_bound(sk, pq, rg, k, max_keep, cs, tid, bar_id, phase);
         }
-        kept = half_walk_kept(pq, rg, L, cs, tid, bar_id, phase, [&](uint64_t x, uint32_t pos) { pq[pos] = x; });
+        kept = half_walk_kept(pq, rg, L, cs, tid, bar_id, phase, pack);
     }
     return L;
 }
 
 // Writes the k best keys of one query's pool (or all, when fewer), unordered,
 // to its output row, then pads the row with (-1, -inf); by the half.  The
-// kept keys are packed to the front of the pool first, so that the row is
-// written with coalesced stores.
+// kept keys are packed first -- into the shared-memory buffer `big` when the
+// pool is in the workspace (k <= 2048 < STREAM_CAND), else to the front of
+// the shared-memory pool -- so that the row is written with coalesced stores.
 __device__ __noinline__ void emit_best(uint64_t* pq, PoolRegions rg, int k, CutScratch& cs, int tid,
                                        uint32_t bar_id, uint32_t& phase, int32_t* out_idx, float* out_score,
                                        uint64_t* big, int big_cap) {
-    auto pack = [&](uint64_t x, uint32_t pos) { pq[pos] = x; };
+    uint64_t* dst = big ? big : pq;
+    auto pack = [&](uint64_t x, uint32_t pos) { dst[pos] = x; };
     const uint32_t ku = static_cast<uint32_t>(k);
     uint32_t out;
     if (rg.total() <= 128 * kRegKeys) {
@@ -831,7 +835,7 @@ __device__ __noinline__ void emit_best(uint64_t* pq, PoolRegions rg, int k, CutS
     bar_sync(bar_id, 128);  // the packed keys are visible to the whole half
     for (int i = tid; i < k; i += 128) {
         if (i < static_cast<int>(out)) {
-            const uint64_t x = pq[i];
+            const uint64_t x = dst[i];
             out_idx[i] = key_index(x);
             out_score[i] = key_score(x);
         } else {
