@@ -283,9 +283,9 @@ si_status si_sort_topk(int32_t* out_idx, float* out_score, int64_t rows, int k, 
     switch (k2 / 32) {
         case 1: si::sort_rows_kernel<1><<<blocks, threads, 0, s>>>(out_idx, out_score, rows, k); break;
         case 2: si::sort_rows_kernel<2><<<blocks, threads, 0, s>>>(out_idx, out_score, rows, k); break;
-        case 4: si::sort_rows_kernel<4><<<blocks, threads, 0, s>>>(out_idx, out_score, rows, k); break;
-        case 8: si::sort_rows_kernel<8><<<blocks, threads, 0, s>>>(out_idx, out_score, rows, k); break;
-        case 16: si::sort_rows_kernel<16><<<blocks, threads, 0, s>>>(out_idx, out_score, rows, k); break;
+        case 4: si::sort_rows_lane_kernel<4><<<blocks, threads, 0, s>>>(out_idx, out_score, rows, k); break;
+        case 8: si::sort_rows_lane_kernel<8><<<blocks, threads, 0, s>>>(out_idx, out_score, rows, k); break;
+        case 16: si::sort_rows_lane_kernel<16><<<blocks, threads, 0, s>>>(out_idx, out_score, rows, k); break;
         case 32: si::sort_rows_block_kernel<1024><<<rows_grid, 128, 0, s>>>(out_idx, out_score, rows, k); break;
         case 64: si::sort_rows_block_kernel<2048><<<rows_grid, 256, 0, s>>>(out_idx, out_score, rows, k); break;
         default: return SI_ERR_UNSUPPORTED;

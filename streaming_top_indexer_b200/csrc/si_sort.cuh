@@ -71,6 +71,88 @@ __global__ void __launch_bounds__(32 * kSortWarps) sort_rows_kernel(int32_t* __r
     }
 }
 
+// Same ordering with E consecutive entries per lane (element i is slot i%E
+// of lane i/E), one warp per row, for E = 4, 8, 16: partner distances below E
+// are register swaps and the rest lane shuffles, fewer shuffle stages than
+// the interleaved layout above, and each lane moves its entries with 16-byte
+// accesses when the row is aligned.
+template <int E>
+__global__ void __launch_bounds__(32 * kSortWarps) sort_rows_lane_kernel(int32_t* __restrict__ idx,
+                                                                         float* __restrict__ score, int64_t rows,
+                                                                         int k) {
+    static_assert(E % 4 == 0 && E <= 16, "four-entry vectors per lane");
+    constexpr int K2 = 32 * E;
+    const int lane = threadIdx.x & 31;
+    const int64_t row = static_cast<int64_t>(blockIdx.x) * kSortWarps + (threadIdx.x >> 5);
+    if (row >= rows) return;
+    int32_t* ri = idx + row * k + lane * E;
+    float* rs = score + row * k + lane * E;
+    const bool vec = ((reinterpret_cast<uintptr_t>(ri) | reinterpret_cast<uintptr_t>(rs)) & 15u) == 0 &&
+                     lane * E + E <= k;
+    uint64_t v[E];
+    if (vec) {
+#pragma unroll
+        for (int c = 0; c < E / 4; ++c) {
+            const int4 i4 = reinterpret_cast<const int4*>(ri)[c];
+            const float4 s4 = reinterpret_cast<const float4*>(rs)[c];
+            v[4 * c + 0] = pack_key(s4.x, static_cast<uint32_t>(i4.x));
+            v[4 * c + 1] = pack_key(s4.y, static_cast<uint32_t>(i4.y));
+            v[4 * c + 2] = pack_key(s4.z, static_cast<uint32_t>(i4.z));
+            v[4 * c + 3] = pack_key(s4.w, static_cast<uint32_t>(i4.w));
+        }
+    } else {
+#pragma unroll
+        for (int e = 0; e < E; ++e)
+            v[e] = (lane * E + e < k) ? pack_key(rs[e], static_cast<uint32_t>(ri[e])) : 0ull;
+    }
+#pragma unroll
+    for (int size = 2; size <= K2; size <<= 1) {
+#pragma unroll
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            if (stride < E) {
+#pragma unroll
+                for (int e = 0; e < E; ++e) {
+                    const int pe = e ^ stride;
+                    if (pe > e) {
+                        const bool desc = ((lane * E + e) & size) == 0;
+                        const uint64_t a = v[e], b = v[pe];
+                        const bool sw = desc ? (a < b) : (a > b);
+                        v[e] = sw ? b : a;
+                        v[pe] = sw ? a : b;
+                    }
+                }
+            } else {
+                const int pl = stride / E;  // partner lane distance
+                const bool lower = (lane & pl) == 0;
+#pragma unroll
+                for (int e = 0; e < E; ++e) {
+                    const uint64_t o = __shfl_xor_sync(0xffffffffu, v[e], pl);
+                    const bool desc = ((lane * E + e) & size) == 0;
+                    const bool take_max = (lower == desc);
+                    v[e] = take_max ? (v[e] > o ? v[e] : o) : (v[e] < o ? v[e] : o);
+                }
+            }
+        }
+    }
+    if (vec) {
+#pragma unroll
+        for (int c = 0; c < E / 4; ++c) {
+            reinterpret_cast<int4*>(ri)[c] = make_int4(key_index(v[4 * c]), key_index(v[4 * c + 1]),
+                                                       key_index(v[4 * c + 2]), key_index(v[4 * c + 3]));
+            reinterpret_cast<float4*>(rs)[c] = make_float4(key_score(v[4 * c]), key_score(v[4 * c + 1]),
+                                                           key_score(v[4 * c + 2]), key_score(v[4 * c + 3]));
+        }
+    } else {
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+            if (lane * E + e < k) {
+                ri[e] = key_index(v[e]);
+                rs[e] = key_score(v[e]);
+            }
+        }
+    }
+}
+
 // Same ordering for long rows (K2 = 1024 or 2048 keys): one block of K2/8
 // threads per row, eight keys per thread; element i is slot i%8 of thread
 // i/8, so each thread loads and stores 8 consecutive entries.  Partner
