@@ -69,3 +69,25 @@ def test_pipelined_host_path_equals_device_call(chunks):
         assert si.check_device_status(bufs["ws"]) == 0
         assert torch.equal(idx_h, ref_idx.cpu())
         assert torch.equal(sc_h.view(torch.int32), ref_sc.cpu().view(torch.int32))
+
+
+def test_windows_with_no_keys_give_padding():
+    B, S, T, H, D, m, k = 2, 600, 0, 64, 128, 4, 8
+    q, w, _ = inputs(B, S, 4, H, D, m, k, seed=5)
+    kc = torch.empty((B, 0, D), dtype=torch.bfloat16, device=DEV)
+    ws = torch.zeros(si.workspace_bytes(B, S, T, H, D, m, k), dtype=torch.uint8, device=DEV)
+    idx = torch.zeros((B, S, k), dtype=torch.int32, device=DEV)
+    sc = torch.zeros((B, S, k), dtype=torch.float32, device=DEV)
+    si.reset_device_status(ws)
+    for t0, t1 in si.host_row_windows(S, 2):
+        si.indexer_topk_rows(q, w, kc, m, k, t0, t1, idx, sc, ws)
+    assert si.check_device_status(ws) == 0
+    assert torch.all(idx == -1) and torch.all(torch.isneginf(sc))
+
+
+def test_reset_clears_a_recorded_timeout():
+    ws = torch.zeros(256, dtype=torch.uint8, device=DEV)
+    assert si.selftest_timeout(ws, limit_ns=5_000_000) == 6  # SI_ERR_TIMEOUT recorded
+    assert si.check_device_status(ws) == 6                    # and kept
+    si.reset_device_status(ws)
+    assert si.check_device_status(ws) == 0
