@@ -5,8 +5,8 @@
  * Streaming Top-k, arXiv 2605.02568v1, Abstract): the lightning indexer of
  * Compressed Sparse Attention scores every compressed key for each query and
  * keeps the top-k keys per query, without materialising the [B,S,H_I,T] fp32
- * score tensor.  The Abstract names the score only "a learned scoring
- * projection over compressed keys"; this library computes
+ * score tensor.  The Abstract gives no formula for the score (only that it is
+ * learned and taken over the compressed keys); this library computes
  *
  *     score[b,t,s] = sum_h w[b,t,h] * max(0, sum_d q[b,t,h,d] * kc[b,s,d])
  *

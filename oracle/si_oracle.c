@@ -9,8 +9,8 @@
  * What it computes (StreamIndex: Memory-Bounded Compressed Sparse Attention
  * via Streaming Top-k, arXiv 2605.02568v1, Abstract): the lightning indexer
  * scores every compressed key for each query, and the k best keys per query
- * are kept.  The Abstract names the score only as "a learned scoring
- * projection over compressed keys"; this library fixes it as
+ * are kept.  The Abstract gives no formula for the score (only that it is
+ * learned and taken over the compressed keys); this library fixes it as
  *
  *     score[b,t,s] = sum_h  w[b,t,h] * max(0, sum_d q[b,t,h,d] * kc[b,s,d])
  *
