@@ -53,6 +53,8 @@ WORKLOADS = {
     "long": Workload("long", 1, 262144, 4, 64, 128, 512),
     "extreme": Workload("extreme", 1, 1048576, 4, 64, 128, 512),
     "tieheavy": Workload("tieheavy", 4, 131072, 4, 64, 128, 2048, "tieheavy"),
+    # the literal reading of the tie-heavy keys: i.i.d. entries from the 16 levels
+    "tieheavy_iid": Workload("tieheavy_iid", 4, 131072, 4, 64, 128, 2048, "tieheavy_iid"),
 }
 
 TIE_LEVELS = [(i - 7.5) / 4.0 for i in range(16)]

@@ -171,7 +171,7 @@ def test_full_size_sampled_rows(name):
 
 
 @pytest.mark.slow
-@pytest.mark.parametrize("name", ["tieheavy", "extreme"])
+@pytest.mark.parametrize("name", ["tieheavy", "tieheavy_iid", "extreme"])
 def test_full_size_sampled_rows_large(name):
     wl = synth.WORKLOADS[name]
     q, w, kc = synth.generate(wl, seed=0, device=DEV)
