@@ -211,10 +211,20 @@ def cpu_baseline(q, w, kc, wl, budget_s: float, seed: int):
     n = int(max(len(probe), min(4096, budget_s / max(per_row, 1e-9))))
     rows = sample_rows_uniform(wl.S, n, seed + 1)
     dt, fl = oracle_sample(q, w, kc, wl, rows)
+    # the same oracle on one host thread, on a sample of about a quarter of the budget
+    n1 = int(max(4, min(len(rows), (budget_s / 4) / max(dt / len(rows) * cores, 1e-9))))
+    rows1 = sample_rows_uniform(wl.S, n1, seed + 2)
+    orc.set_threads(1)
+    try:
+        dt1, fl1 = oracle_sample(q, w, kc, wl, rows1)
+    finally:
+        orc.set_threads(cores)
     return {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
             "rows_per_s": len(rows) / dt,
+            "value_1thread": fl1 / dt1 / 1e12, "rows_per_s_1thread": len(rows1) / dt1,
             "sample": f"{len(rows)} uniformly sampled query rows of batch 0 of the {wl.name} workload "
-                      f"(fp64 C oracle, OpenMP, {dt:.1f} s)"}
+                      f"(fp64 C oracle, OpenMP, {dt:.1f} s); one-thread figure on {len(rows1)} rows "
+                      f"({dt1:.1f} s)"}
 
 
 def run_reference(args, world, rank, local):
@@ -272,6 +282,7 @@ def run_ours(args, world, rank, local):
     wl = synth.WORKLOADS[args.workload]
     B, S, T, H, D, m, k = wl.B, wl.S, wl.T, wl.H, wl.D, wl.m, wl.k
     torch.cuda.reset_peak_memory_stats(dev)
+    free0 = torch.cuda.mem_get_info(dev)[0]
     q, w, kc = synth.generate(wl, seed=args.seed + rank, device=dev)
     idx = torch.empty((B, S, k), dtype=torch.int32, device=dev)
     sc = torch.empty((B, S, k), dtype=torch.float32, device=dev)
@@ -306,6 +317,9 @@ def run_ours(args, world, rank, local):
     select_ms = [e[0].elapsed_time(e[1]) for e in ev]
     sort_ms = [e[1].elapsed_time(e[2]) for e in ev]
     peak_bytes = torch.cuda.max_memory_allocated(dev)
+    # cross-check: device memory taken since the start, as the driver sees it
+    # (the caching allocator's reservations included)
+    mem_get_info_bytes = free0 - torch.cuda.mem_get_info(dev)[0]
     total_ms_max = all_max(total_ms, world, dev)
 
     pairs = visible_pairs(B, S, T, m)
@@ -329,6 +343,7 @@ def run_ours(args, world, rank, local):
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_of(wl, args),
             "rows_per_s": rows_per_s, "peak_hbm_bytes": int(peak_bytes), "peak_hbm_gb": peak_bytes / 1e9,
+            "hbm_taken_mem_get_info_bytes": int(mem_get_info_bytes),
             "workspace_bytes": ws_bytes, "gpu_launches": 2 * args.steps, "roofline": roofline,
             "clocks": sampler.summary()}
 
