@@ -43,7 +43,7 @@ __global__ void __launch_bounds__(32 * kSortWarps) sort_rows_kernel(int32_t* __r
                     if (pe > e) {
                         const bool desc = ((e * 32) & size) == 0;
                         const uint64_t a = v[e], b = v[pe];
-                        const bool swap = desc ? (a < b) : (a > b);
+                        const bool swap = (a < b) == desc;  // keys distinct, or equal padding
                         v[e] = swap ? b : a;
                         v[pe] = swap ? a : b;
                     }
@@ -56,7 +56,7 @@ __global__ void __launch_bounds__(32 * kSortWarps) sort_rows_kernel(int32_t* __r
                     const bool lower = (lane & stride) == 0;
                     const bool desc = (i & size) == 0;
                     const bool take_max = (lower == desc);
-                    v[e] = take_max ? (v[e] > other ? v[e] : other) : (v[e] < other ? v[e] : other);
+                    v[e] = ((v[e] > other) == take_max) ? v[e] : other;
                 }
             }
         }
@@ -114,9 +114,11 @@ __global__ void __launch_bounds__(32 * kSortWarps) sort_rows_lane_kernel(int32_t
                 for (int e = 0; e < E; ++e) {
                     const int pe = e ^ stride;
                     if (pe > e) {
+                        // keys are distinct (padding zeros are equal, and swapping
+                        // them changes nothing), so one compare decides
                         const bool desc = ((lane * E + e) & size) == 0;
                         const uint64_t a = v[e], b = v[pe];
-                        const bool sw = desc ? (a < b) : (a > b);
+                        const bool sw = (a < b) == desc;
                         v[e] = sw ? b : a;
                         v[pe] = sw ? a : b;
                     }
@@ -129,7 +131,7 @@ __global__ void __launch_bounds__(32 * kSortWarps) sort_rows_lane_kernel(int32_t
                     const uint64_t o = __shfl_xor_sync(0xffffffffu, v[e], pl);
                     const bool desc = ((lane * E + e) & size) == 0;
                     const bool take_max = (lower == desc);
-                    v[e] = take_max ? (v[e] > o ? v[e] : o) : (v[e] < o ? v[e] : o);
+                    v[e] = ((v[e] > o) == take_max) ? v[e] : o;
                 }
             }
         }
@@ -202,7 +204,7 @@ __global__ void __launch_bounds__(K2 / 8) sort_rows_block_kernel(int32_t* __rest
                     if (pe > e) {
                         const bool desc = ((tid * E + e) & size) == 0;
                         const uint64_t a = v[e], b = v[pe];
-                        const bool sw = desc ? (a < b) : (a > b);
+                        const bool sw = (a < b) == desc;  // keys distinct, or equal padding
                         v[e] = sw ? b : a;
                         v[pe] = sw ? a : b;
                     }
@@ -226,7 +228,7 @@ __global__ void __launch_bounds__(K2 / 8) sort_rows_block_kernel(int32_t* __rest
                 for (int e = 0; e < E; ++e) {
                     const bool desc = ((tid * E + e) & size) == 0;
                     const bool take_max = (lower == desc);
-                    v[e] = take_max ? (v[e] > o[e] ? v[e] : o[e]) : (v[e] < o[e] ? v[e] : o[e]);
+                    v[e] = ((v[e] > o[e]) == take_max) ? v[e] : o[e];
                 }
             }
         }
