@@ -44,7 +44,10 @@ def check_against_oracle(q, w, kc, m, k, b_rows, t_rows, g_idx=None, g_score=Non
     gi = g_idx[bt, tt].cpu().numpy()
     gs = g_score[bt, tt].cpu().numpy()
     o_idx, o_score, o_meta, o_scores = oracle_rows(q, w, kc, m, k, b_rows, t_rows)
-    return checker.check_rows(gi, gs, o_idx, o_score, o_meta, o_scores, k, where)
+    bound = checker.score_error_bound(synth.bf16_bits(q[bt.to(q.device), tt.to(q.device)]),
+                                      w[bt.to(w.device), tt.to(w.device)].cpu().numpy(), synth.bf16_bits(kc),
+                                      b_rows, gi)
+    return checker.check_rows(gi, gs, o_idx, o_score, o_meta, o_scores, k, bound, where)
 
 
 def all_rows(B, S):

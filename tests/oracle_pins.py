@@ -74,7 +74,10 @@ def check_invariants(idx, score, nvis, k):
 # --------------------------------------------------------------------------
 
 def pin_hand_cases(lib):
-    """Hand-computed fixtures under tests/golden/."""
+    """Hand-computed fixtures under tests/golden/: indices, scores and the
+    per-row meta (max |score| over the visible keys, the scores at ranks k
+    and k+1, the visible count) that the acceptance rule's tie band and
+    score tolerance are built on."""
     for name in sorted(os.listdir(GOLDEN)):
         if not name.startswith("hand_case_"):
             continue
@@ -84,11 +87,13 @@ def pin_hand_cases(lib):
         q = f32_to_bf16_bits(case["q"]).reshape(B, S, H, D)
         w = np.asarray(case["w"], np.float32).reshape(B, S, H)
         kc = f32_to_bf16_bits(case["kc"]).reshape(B, T, D)
-        idx, sc, _, _ = run_all(lib, q, w, kc, m, k)
+        idx, sc, meta, _ = run_all(lib, q, w, kc, m, k)
         e_idx = np.asarray(case["expect_idx"], np.int32).reshape(B, S, k)
         e_sc = np.asarray([[float(v) for v in row] for row in case["expect_score"]]).reshape(B, S, k)
         assert np.array_equal(idx, e_idx), f"{name}: idx {idx.tolist()} != {e_idx.tolist()}"
         assert np.array_equal(sc, e_sc), f"{name}: score {sc.tolist()} != {e_sc.tolist()}"
+        e_meta = np.asarray([[float(v) for v in row] for row in case["expect_meta"]]).reshape(B, S, 4)
+        assert np.array_equal(meta, e_meta, equal_nan=True), f"{name}: meta {meta.tolist()} != {e_meta.tolist()}"
 
 
 def pin_matmul_special_case(lib, seed=1):

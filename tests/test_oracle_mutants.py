@@ -24,6 +24,13 @@ MUTANTS = {
     "last_head_dropped": ("for (int h = 0; h < H; ++h) {", "for (int h = 0; h < H - 1; ++h) {"),
     "padding_score_zero": ("out_score[r * k + j] = -INFINITY;", "out_score[r * k + j] = 0.0;"),
     "w_of_wrong_head": ("score += (double)w_row[h] * relu;", "score += (double)w_row[H - 1 - h] * relu;"),
+    # the per-row meta that the acceptance rule's tie band and tolerance use
+    "rank_k_off_by_one": ("(k - 1 < nvis) ? keys[k - 1].score : NAN", "(k < nvis) ? keys[k].score : NAN"),
+    "rank_k1_off_by_one": ("(k < nvis) ? keys[k].score : NAN", "(k + 1 < nvis) ? keys[k + 1].score : NAN"),
+    "rowmax_signed": ("if (fabs(sc) > rowmax) rowmax = fabs(sc);", "if (sc > rowmax) rowmax = sc;"),
+    "rowmax_over_invisible_keys": (
+        "if (fabs(sc) > rowmax) rowmax = fabs(sc);\n            }",
+        "}\n            { double a = fabs(indexer_score(q_row, w_row, kc_b + s * D, H, D)); if (a > rowmax) rowmax = a; }"),
 }
 
 

@@ -27,18 +27,20 @@ def test_pin(lib, pin):
 ])
 def test_c_oracle_matches_numpy_restatement(lib, B, S, m, H, D, k, Tover):
     """The C oracle and an independent numpy restatement agree exactly on
-    indices and to fp64 rounding on scores."""
+    indices and to fp64 rounding on scores and on the per-row meta."""
     rng = np.random.default_rng(S * 31 + k)
     T = S // m if Tover is None else Tover
     q = pins.random_bf16(rng, (B, S, H, D), scale=1 / np.sqrt(D))
     w = rng.standard_normal((B, S, H)).astype(np.float32)
     kc = pins.random_bf16(rng, (B, T, D))
-    idx, sc, _, _ = orc.topk_all_rows(q, w, kc, m, k, lib=lib)
-    bidx, bsc = brute.topk_all_rows(q, w, kc, m, k)
+    idx, sc, meta, _ = orc.topk_all_rows(q, w, kc, m, k, lib=lib)
+    bidx, bsc, bmeta = brute.topk_all_rows(q, w, kc, m, k, with_meta=True)
     assert np.array_equal(idx, bidx)
     fin = np.isfinite(bsc)
     assert np.array_equal(np.isfinite(sc), fin)
     assert np.allclose(sc[fin], bsc[fin], rtol=1e-12, atol=1e-12)
+    assert np.array_equal(np.isnan(meta), np.isnan(bmeta))
+    assert np.allclose(meta, bmeta, rtol=1e-12, atol=1e-12, equal_nan=True)
 
 
 def test_materialised_size_formula():
