@@ -158,10 +158,16 @@ SI_API si_status si_selftest_timeout(void* workspace, size_t workspace_bytes, ui
  * start at zero.  Calls whose work overlaps on the GPU (different streams,
  * no ordering between them) race on the shared array: order them.
  *
- * Limit: configurations whose si_workspace_bytes() exceeds 1 MiB -- those
- * whose candidate pools do not fit in shared memory, e.g. k > 512 at
- * H_I=64, d_I=128 -- return SI_ERR_WORKSPACE_TOO_SMALL before anything is
- * enqueued.  Everything else is as si_indexer_topk.  out_status, if not NULL,
+ * Limit: configurations whose si_workspace_bytes() exceeds 1 MiB return
+ * SI_ERR_WORKSPACE_TOO_SMALL before anything is enqueued.  Those are exactly
+ * the ones whose candidate pools do not fit in shared memory.  The first
+ * refused k for each (H_I, d_I) is:
+ *     H_I=64: d_I=128 k >= 1089; d_I=64 none (every k up to 2048 runs)
+ *     H_I=32: d_I=128 k >= 465;  d_I=64 k >= 1185
+ *     H_I=16: d_I=128 k >= 161;  d_I=64 k >= 481
+ *     H_I=8:  d_I=128 every k;   d_I=64 k >= 193
+ * So the array only ever holds the device error word.  Everything else is
+ * as si_indexer_topk.  out_status, if not NULL,
  * is a device word that receives the device status of the call (0, or
  * SI_ERR_TIMEOUT) once the stream reaches the end of the call. */
 SI_API si_status si_indexer_topk_noalloc(const void* q, const float* w, const void* kc,

@@ -15,7 +15,8 @@ compression ratio m=4):
   extreme   B=1 S=1048576   T=262144  H_I=64 d_I=128 k=512
   tieheavy  B=4 S=131072    T=32768   H_I=64 d_I=128 k=2048  (16-level keys)
 
-q is N(0,1) scaled by 1/sqrt(d_I) in fp32 and then rounded once to bf16; kc
+q is N(0,1) scaled by 1/sqrt(d_I) in fp32 and then rounded once to bf16
+(drawn in fixed blocks of rows, so generation needs no full fp32 copy); kc
 is N(0,1) rounded to bf16; w is fp32 N(0,1)/sqrt(H_I).  The tie-heavy
 workload draws a 16-row codebook per batch whose entries come from the 16
 bf16-exact levels (i-7.5)/4, i=0..15, and copies a uniformly chosen codebook
@@ -59,6 +60,10 @@ WORKLOADS = {
 
 TIE_LEVELS = [(i - 7.5) / 4.0 for i in range(16)]
 
+# fp32 values of q drawn per block (256 MiB); fixed, so that a seed names the
+# same inputs on every run.
+Q_BLOCK_ELEMS = 1 << 26
+
 
 def generate(wl: Workload, seed: int = 0, device="cpu", T: int | None = None):
     """Draw (q bf16 [B,S,H,D], w fp32 [B,S,H], kc bf16 [B,T,D]) for a workload.
@@ -69,10 +74,18 @@ def generate(wl: Workload, seed: int = 0, device="cpu", T: int | None = None):
     dev = torch.device(device)
     g = torch.Generator(device=dev)
     g.manual_seed(seed)
-    q = torch.randn((wl.B, wl.S, wl.H, wl.D), generator=g, device=dev,
-                    dtype=torch.float32)
-    q.mul_(1.0 / math.sqrt(wl.D))
-    q = q.to(torch.bfloat16)
+    # q is drawn in fp32 blocks of at most Q_BLOCK_ELEMS values, each scaled
+    # and rounded to bf16 in place, so no full-size fp32 copy ever exists
+    # (at S=1,048,576 that copy alone would be 34 GB).
+    q = torch.empty((wl.B, wl.S, wl.H, wl.D), dtype=torch.bfloat16, device=dev)
+    rows = max(1, Q_BLOCK_ELEMS // (wl.H * wl.D))
+    for b in range(wl.B):
+        for s0 in range(0, wl.S, rows):
+            s1 = min(wl.S, s0 + rows)
+            blk = torch.randn((s1 - s0, wl.H, wl.D), generator=g, device=dev, dtype=torch.float32)
+            blk.mul_(1.0 / math.sqrt(wl.D))
+            q[b, s0:s1].copy_(blk)
+            del blk
     if wl.kind.startswith("tieheavy"):
         w = torch.rand((wl.B, wl.S, wl.H), generator=g, device=dev,
                        dtype=torch.float32)
