@@ -4,9 +4,9 @@
                     [--workload long] [--no-e2e] [--no-cpu-baseline]
     python bench.py --sweep k|s [--workload v4flash] [--sweep-values ...]
 
-A step is one indexer call over one batch of synthetic inputs: the fused
-scoring + selection kernel and the per-row sort (what si_indexer_topk
-launches), with q, w, kc already resident in HBM.  Every rank runs its own
+A step is one si_indexer_topk call over one batch of synthetic inputs: the
+fused scoring, selection and row-sort kernel, with q, w, kc already resident
+in HBM.  Every rank runs its own
 problem of the named workload (seeds differ by rank), so per-GPU work is
 fixed as N grows ("scaling": "weak"); no data moves between ranks.
 
@@ -295,32 +295,36 @@ def run_ours(args, world, rank, local):
     ws = torch.zeros(ws_bytes, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
+    if args.sort_kernel:
+        si.set_sort_in_select(False)  # the earlier design: unordered rows + the row-sort kernel
+    sorted_in_select = si.select_sorts_rows(H, D, k)
+    launches_per_step = 1 if sorted_in_select else 2
+
+    # One step is the product call, si_indexer_topk: a 256-byte reset of the
+    # workspace header, then the select kernel (which also sorts the rows),
+    # plus the row-sort kernel only where the select kernel cannot sort.
     def step():
-        si.select_topk(q, w, kc, m, k, idx, sc, ws, stream)
-        si.sort_topk(idx, sc, stream)
+        si.indexer_topk(q, w, kc, m, k, idx, sc, ws, stream)
 
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize(dev)
     assert si.check_device_status(ws) == 0, "device error during warm-up"
 
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
     sampler = ClockSampler(local)
     with sampler:
         barrier(world)
         torch.cuda.synchronize(dev)
         for i in range(args.steps):
             ev[i][0].record(stream)
-            si.select_topk(q, w, kc, m, k, idx, sc, ws, stream)
+            step()
             ev[i][1].record(stream)
-            si.sort_topk(idx, sc, stream)
-            ev[i][2].record(stream)
         torch.cuda.synchronize(dev)
         barrier(world)
     assert si.check_device_status(ws) == 0, "device error during the timed region"
-    total_ms = ev[0][0].elapsed_time(ev[-1][2])
-    select_ms = [e[0].elapsed_time(e[1]) for e in ev]
-    sort_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    total_ms = ev[0][0].elapsed_time(ev[-1][1])
+    call_ms = [e[0].elapsed_time(e[1]) for e in ev]
     peak_bytes = torch.cuda.max_memory_allocated(dev)
     # cross-check: device memory taken by the outputs and workspace, as the
     # driver sees it (the caching allocator's rounding included)
@@ -335,15 +339,20 @@ def run_ours(args, world, rank, local):
     rows_per_s = world * B * S * args.steps / (total_ms_max * 1e-3)
 
     peaks, peak_src = load_peaks()
-    sel_avg_ms = statistics.mean(select_ms)
-    achieved = flops_rank / (sel_avg_ms * 1e-3) / 1e12
+    # The dominant kernel's duration: each call's events bracket the 256-byte
+    # header reset (a few microseconds) and the select kernel, and also the
+    # row sort where the select kernel leaves rows unordered.  So this slightly
+    # understates the kernel's own rate.
+    call_avg_ms = statistics.mean(call_ms)
+    achieved = flops_rank / (call_avg_ms * 1e-3) / 1e12
     traffic = ncu_traffic(wl.name)
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                 "frac": achieved / peaks["bf16_tflops"], "traffic": traffic,
                 "peak_source": f"{peak_src} bf16 burst",
                 "frac_of_sustained": achieved / peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]),
-                "kernel": "select_kernel<64,128>" if (H, D) == (64, 128) else f"select_kernel<{H},{D}>",
-                "select_ms": sel_avg_ms, "sort_ms": statistics.mean(sort_ms)}
+                "kernel": f"select_kernel<{H},{D}>",
+                "kernel_ms": call_avg_ms, "kernel_ms_scope": "whole si_indexer_topk call",
+                "rows_sorted_in_select": sorted_in_select}
 
     line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
@@ -359,7 +368,7 @@ def run_ours(args, world, rank, local):
                                     "workspace": int(ws_bytes),
                                     "outputs_workspace_mem_get_info": int(mem_get_info_bytes)},
             "peak_hbm_scope": "allocator peak during the indexer calls, inputs resident, input generation excluded",
-            "workspace_bytes": ws_bytes, "gpu_launches": 2 * args.steps, "roofline": roofline,
+            "workspace_bytes": ws_bytes, "gpu_launches": launches_per_step * args.steps, "roofline": roofline,
             "clocks": sampler.summary()}
 
     # end to end through the public API with host buffers
@@ -415,30 +424,32 @@ def run_sweep(args):
             dense = si.indexer_scores(q, w, kc, m)[0] if S * T * 4 <= args.sweep_dense_bytes else None
             dense_cache[S] = (q, w, kc, dense)
         q, w, kc, dense = dense_cache[S]
+        torch.cuda.synchronize(dev)
+        torch.cuda.reset_peak_memory_stats(dev)
+        base_bytes = torch.cuda.memory_allocated(dev)  # inputs (and the cached dense scores)
         idx = torch.empty((B, S, k), dtype=torch.int32, device=dev)
         sc = torch.empty((B, S, k), dtype=torch.float32, device=dev)
         ws = torch.zeros(si.workspace_bytes(B, S, T, H, D, m, k), dtype=torch.uint8, device=dev)
         for _ in range(args.warmup):
-            si.select_topk(q, w, kc, m, k, idx, sc, ws, stream)
-            si.sort_topk(idx, sc, stream)
+            si.indexer_topk(q, w, kc, m, k, idx, sc, ws, stream)
         torch.cuda.synchronize(dev)
-        e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
-        sel, srt = [], []
+        e0, e1 = (torch.cuda.Event(enable_timing=True) for _ in range(2))
+        times = []
         for _ in range(args.steps):
             e0.record(stream)
-            si.select_topk(q, w, kc, m, k, idx, sc, ws, stream)
+            si.indexer_topk(q, w, kc, m, k, idx, sc, ws, stream)
             e1.record(stream)
-            si.sort_topk(idx, sc, stream)
-            e2.record(stream)
             torch.cuda.synchronize(dev)
-            sel.append(e0.elapsed_time(e1))
-            srt.append(e1.elapsed_time(e2))
+            times.append(e0.elapsed_time(e1))
         assert si.check_device_status(ws) == 0, "device error in the sweep"
         flops = 2.0 * H * D * visible_pairs(B, S, T, m)
-        ms = statistics.median(sel) + statistics.median(srt)
+        ms = statistics.median(times)
+        inputs = q.numel() * 2 + w.numel() * 4 + kc.numel() * 2
+        # indexer footprint: inputs + outputs + workspace (the dense scores of the recall check excluded)
+        peak_idx = inputs + torch.cuda.max_memory_allocated(dev) - base_bytes
         cell = {"sweep": args.sweep, "workload": base.name, "B": B, "S": S, "T": T, "H_I": H, "d_I": D, "m": m,
-                "k": k, "value": flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "select_ms": statistics.median(sel),
-                "sort_ms": statistics.median(srt), "steps": args.steps, "warmup": args.warmup,
+                "k": k, "value": flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms": ms,
+                "steps": args.steps, "warmup": args.warmup, "peak_hbm_bytes": int(peak_idx),
                 "recall_vs_materialised": None}
         if dense is not None:
             g = torch.Generator().manual_seed(args.seed + 1)
@@ -499,6 +510,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sort-kernel", action="store_true",
+                    help="sort rows in the separate row-sort kernel instead of inside the select kernel")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work")
     ap.add_argument("--ref-budget", type=float, default=60.0, help="seconds of oracle work, reference arm")
     ap.add_argument("--sweep", choices=["k", "s"], default=None,

@@ -67,9 +67,10 @@ typedef enum {
 SI_API size_t si_workspace_bytes(int64_t B, int64_t S, int64_t T, int H_I, int d_I, int m, int k);
 
 /* The indexer step: top-k keys and scores of every query row.
- * Enqueues: a 256-byte reset of the workspace header, the fused scoring and
- * selection kernel, and the per-row sort.  Writes every element of out_idx
- * and out_score, padding included. */
+ * Enqueues: a 256-byte reset of the workspace header, then the fused scoring,
+ * selection and row-sort kernel.  The separate per-row sort is added only
+ * where si_select_sorts_rows() is 0.  Writes every element of out_idx and
+ * out_score, padding included. */
 SI_API si_status si_indexer_topk(const void* q, const float* w, const void* kc,
                           int64_t B, int64_t S, int64_t T, int H_I, int d_I, int m, int k,
                           int32_t* out_idx, float* out_score,
@@ -100,16 +101,20 @@ SI_API si_status si_indexer_topk_rows(const void* q, const float* w, const void*
                                void* workspace, size_t workspace_bytes, si_stream_t stream);
 
 /* First stage of si_indexer_topk alone: the fused scoring + selection kernel.
- * Leaves each row's top-k set in out_idx/out_score unordered (padding at the
- * tail).  Does not reset the workspace header.  Exposed so that the stages
- * can be timed separately; si_indexer_topk == header reset + this + sort. */
+ * Does not reset the workspace header.  Where si_select_sorts_rows() is 1
+ * for these sizes, the kernel also sorts each row at the end of its work
+ * unit, and the rows are final.  Otherwise each row's top-k set is left
+ * unordered (padding at the tail) for si_sort_topk.  Exposed so that the
+ * stages can be timed separately: si_indexer_topk is the header reset, then
+ * this, then si_sort_topk only where the kernel leaves rows unordered. */
 SI_API si_status si_select_topk(const void* q, const float* w, const void* kc,
                          int64_t B, int64_t S, int64_t T, int H_I, int d_I, int m, int k,
                          int32_t* out_idx, float* out_score,
                          void* workspace, size_t workspace_bytes, si_stream_t stream);
 
 /* Second stage: orders each of the `rows` rows of k (index, score) pairs by
- * score descending, then index ascending, padding last (in place). */
+ * score descending, then index ascending, padding last (in place).  Also a
+ * general utility for rows in any order. */
 SI_API si_status si_sort_topk(int32_t* out_idx, float* out_score, int64_t rows, int k,
                        si_stream_t stream);
 
@@ -174,6 +179,20 @@ SI_API si_status si_indexer_topk_noalloc(const void* q, const float* w, const vo
                                          int64_t B, int64_t S, int64_t T, int H_I, int d_I, int m, int k,
                                          int32_t* out_idx, float* out_score, uint32_t* out_status,
                                          si_stream_t stream);
+
+/* 1 if the select kernel writes rows already sorted for these sizes: every
+ * k <= 1024.  The kernel's unit-end sort covers 128*E keys, with E the
+ * smallest power of two such that 128*E >= k.  For larger k the separate
+ * row sort is faster.  Otherwise 0, and si_indexer_topk adds the si_sort_topk
+ * pass.
+ * Host arithmetic only.  Returns 0 for unsupported sizes. */
+SI_API int si_select_sorts_rows(int H_I, int d_I, int k);
+
+/* Process-wide switch for later calls.  Nonzero (the default): the select
+ * kernel sorts rows where it can.  Zero: it always leaves rows unordered,
+ * and si_indexer_topk sorts them with the separate row-sort kernel.  Both give
+ * identical results; the switch exists to time the two designs. */
+SI_API void si_set_sort_in_select(int enable);
 
 /* Device-side wait limit, in nanoseconds, used by later calls (default 2 s). */
 SI_API void si_set_timeout_ns(uint64_t ns);

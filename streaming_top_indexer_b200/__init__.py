@@ -22,7 +22,8 @@ import torch
 __all__ = [
     "SIError", "library_path", "load_library", "workspace_bytes", "indexer_topk",
     "select_topk", "sort_topk", "indexer_scores", "check_device_status",
-    "selftest_timeout", "set_timeout_ns", "indexer_topk_host", "version",
+    "selftest_timeout", "set_timeout_ns", "indexer_topk_host", "version", "select_sorts_rows",
+    "set_sort_in_select",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -67,6 +68,10 @@ def _declare(lib):
     lib.si_selftest_timeout.argtypes = [vp, sz, c.c_uint64, vp]
     lib.si_set_timeout_ns.restype = None
     lib.si_set_timeout_ns.argtypes = [c.c_uint64]
+    lib.si_select_sorts_rows.restype = c.c_int
+    lib.si_select_sorts_rows.argtypes = [i32, i32, i32]
+    lib.si_set_sort_in_select.restype = None
+    lib.si_set_sort_in_select.argtypes = [i32]
     lib.si_status_string.restype = c.c_char_p
     lib.si_status_string.argtypes = [c.c_int]
     lib.si_version.restype = c.c_char_p
@@ -91,6 +96,18 @@ def version() -> str:
 
 def set_timeout_ns(ns: int) -> None:
     load_library().si_set_timeout_ns(int(ns))
+
+
+def select_sorts_rows(H: int, D: int, k: int) -> bool:
+    """Whether the select kernel writes rows already sorted for these sizes
+    (si_select_sorts_rows); otherwise indexer_topk adds the row-sort kernel."""
+    return bool(load_library().si_select_sorts_rows(int(H), int(D), int(k)))
+
+
+def set_sort_in_select(enable: bool) -> None:
+    """Process-wide: sort rows inside the select kernel (default) or always
+    in the separate row-sort kernel (si_set_sort_in_select)."""
+    load_library().si_set_sort_in_select(1 if enable else 0)
 
 
 def _stream(stream):
@@ -189,7 +206,8 @@ def indexer_topk_rows(q, w, kc, m: int, k: int, t_begin: int, t_end: int, out_id
 
 
 def select_topk(q, w, kc, m: int, k: int, out_idx=None, out_score=None, workspace=None, stream=None):
-    """First stage only (si_select_topk): each row's top-k set, unordered."""
+    """First stage only (si_select_topk): each row's top-k set, already in
+    final order where select_sorts_rows(H, D, k), else unordered."""
     return _topk_call("si_select_topk", q, w, kc, m, k, out_idx, out_score, workspace, stream)
 
 

@@ -14,12 +14,11 @@
 #include <mutex>
 
 #include "si.h"
-#include "si_ptx.cuh"
+#include "si_host.cuh"
 #include "si_keys.cuh"
-#include "si_select.cuh"
 #include "si_sort.cuh"
 
-namespace {
+namespace si_host {
 
 // With SI_DEBUG set in the environment, CUDA failures are also printed to stderr.
 si_status cuda_fail(const char* where, cudaError_t e) {
@@ -28,15 +27,68 @@ si_status cuda_fail(const char* where, cudaError_t e) {
     return SI_ERR_CUDA;
 }
 
-constexpr int kMaxCtas = 148;                 // persistent CTAs (one per B200 SM)
-constexpr size_t kHeaderBytes = 256;          // error word + reserved
+namespace {
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+}  // namespace
+
+bool encode_3d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t d0, uint64_t d1,
+               uint64_t d2, uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t box0, uint32_t box1,
+               CUtensorMapSwizzle sw) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {d0, d1, d2};
+    cuuint64_t strides[2] = {stride1_bytes, stride2_bytes};
+    cuuint32_t box[3] = {box0, box1, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    std::memset(map, 0, sizeof(*map));
+    CUresult r = enc(map, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+namespace {
+std::mutex g_dev_mu;
+int g_dev_sms[64] = {};
+}  // namespace
+
+int device_sms(int dev) {
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    if (dev < 0 || dev >= 64) return 0;
+    if (g_dev_sms[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+        g_dev_sms[dev] = n;
+    }
+    return g_dev_sms[dev];
+}
+
+}  // namespace si_host
+
+namespace {
+
+using si_host::cuda_fail;
+using si_host::kHeaderBytes;
+using si_host::kMaxCtas;
+using si_host::kMaxDynSmem;
 // Row windows of si_indexer_topk_rows start (and, except at S, end) on
 // multiples of this, a multiple of every unit's query count (256/H_I).
 constexpr int64_t kRowAlign = 256;
-constexpr uint32_t kMaxDynSmem = 232448;      // 227 KB opt-in per block on sm_100
-constexpr uint32_t kMinDynSmem = 120 * 1024;  // > half an SM: one CTA per SM, so
-                                              // two CTAs never compete for TMEM
 std::atomic<uint64_t> g_timeout_ns{2000000000ull};
+// Whether the select kernel sorts each row at unit end (default) or leaves the
+// rows unordered for the separate row sort.
+std::atomic<bool> g_sort_in_select{true};
 
 bool supported_h(int h) { return h == 8 || h == 16 || h == 32 || h == 64; }
 bool supported_d(int d) { return d == 64 || d == 128; }
@@ -78,6 +130,30 @@ PoolPlan pool_plan(int H, int D, int k) {
     return {false, r32(4 * k > k + 288 ? 4 * k : k + 288)};
 }
 
+// Keys per thread of the unit-end row sort inside the select kernel (the
+// half's 128 threads sort 128 * E >= k keys), or 0 when rows are left
+// unordered for the separate row-sort kernel:
+//  - k > 1024 (E = 16): the network no longer unrolls into registers, and
+//    measured at k = 2048 (B=4, S=131,072) the select kernel then took 407 ms
+//    against 205 ms + 22.5 ms for the separate sort;
+//  - the sort's exchange buffer (the query's own shared-memory pool, or the
+//    half's STREAM_CAND-key buffer with workspace pools) holds fewer than
+//    128 * E keys.
+// At k = 512 (S=262,144) the two designs measured within 0.5 % of each other.
+int row_sort_e(int H, int D, int k) {
+    if (k > 1024) return 0;
+    int e = 1;
+    while (128 * e < k) e <<= 1;
+    const PoolPlan pp = pool_plan(H, D, k);
+    int cap = 0;
+#define SI_CASE(HH, DD) \
+    if (H == HH && D == DD) cap = pp.smem ? pp.P : si::SelCfg<HH, DD>::STREAM_CAND;
+    SI_CASE(8, 64) SI_CASE(8, 128) SI_CASE(16, 64) SI_CASE(16, 128)
+    SI_CASE(32, 64) SI_CASE(32, 128) SI_CASE(64, 64) SI_CASE(64, 128)
+#undef SI_CASE
+    return 128 * e <= cap ? e : 0;
+}
+
 size_t global_pool_bytes(int H, int D, int k) {
     const PoolPlan pp = pool_plan(H, D, k);
     if (pp.smem) return 0;
@@ -111,132 +187,53 @@ si_status check_topk(const void* q, const float* w, const void* kc, int64_t B, i
     return SI_OK;
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    });
-    return fn;
-}
-
-bool encode_3d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t d0, uint64_t d1,
-               uint64_t d2, uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t box0, uint32_t box1,
-               CUtensorMapSwizzle sw) {
-    auto enc = tensor_map_encoder();
-    if (!enc) return false;
-    cuuint64_t dims[3] = {d0, d1, d2};
-    cuuint64_t strides[2] = {stride1_bytes, stride2_bytes};
-    cuuint32_t box[3] = {box0, box1, 1};
-    cuuint32_t estr[3] = {1, 1, 1};
-    std::memset(map, 0, sizeof(*map));
-    CUresult r = enc(map, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                     sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
-}
-
-struct DeviceInfo {
-    int sms = 0;
-    bool attr_set[2][4][2] = {};  // [D==128][log2(H/8)][unused]
-};
-
-std::mutex g_dev_mu;
-DeviceInfo g_dev[64];
-
-int device_sms(int dev) {
-    std::lock_guard<std::mutex> lk(g_dev_mu);
-    if (dev < 0 || dev >= 64) return 0;
-    if (g_dev[dev].sms == 0) {
-        int n = 0;
-        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-        g_dev[dev].sms = n;
-    }
-    return g_dev[dev].sms;
-}
-
-template <int H, int D>
-si_status launch_select_t(const void* q, const float* w, const void* kc, int64_t B, int64_t S, int64_t T, int m,
-                          int k, int32_t* out_idx, float* out_score, float* dense, void* ws, cudaStream_t stream,
-                          int64_t t_lo, int64_t t_hi) {
-    using C = si::SelCfg<H, D>;
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return SI_ERR_CUDA;
-    const int sms = device_sms(dev);
-    if (sms <= 0) return SI_ERR_CUDA;
-
-    si::SelectParams p{};
-    p.B = B;
-    p.S = S;
-    p.T = T;
-    p.m = m;
-    p.k = dense ? 1 : k;
-    const PoolPlan pp = dense ? PoolPlan{true, 0} : pool_plan(H, D, p.k);
-    p.P = pp.P;
-    p.t_lo = t_lo;
-    p.t_hi = t_hi;
-    p.nblk = (t_hi - t_lo + C::QT - 1) / C::QT;
-    p.units = B * p.nblk;
-    p.out_idx = out_idx;
-    p.out_score = out_score;
-    p.dense = dense;
-    p.err = static_cast<uint32_t*>(ws);
-    p.timeout_ns = g_timeout_ns.load();
-    const bool smem_pool = pp.smem;
-    p.gpool = smem_pool ? nullptr
-                        : reinterpret_cast<uint64_t*>(static_cast<uint8_t*>(ws) + kHeaderBytes);
-#ifdef SI_TRACE
-    // Tracing builds: per-warp cycle counters after the pools; the caller adds
-    // kMaxCtas * kTraceWarps * kTraceSlots * 8 bytes to the workspace.
-    p.trace = reinterpret_cast<unsigned long long*>(static_cast<uint8_t*>(ws) + kHeaderBytes +
-                                                    (smem_pool ? 0 : global_pool_bytes(H, D, p.k)));
-#endif
-
-    CUtensorMap tq, tkc, tw;
-    const uint64_t bf = 2;
-    if (!encode_3d(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q, D, static_cast<uint64_t>(S) * H, B, D * bf,
-                   static_cast<uint64_t>(S) * H * D * bf, 64, C::N, CU_TENSOR_MAP_SWIZZLE_128B))
-        return SI_ERR_CUDA;
-    if (!encode_3d(&tkc, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kc, D, T, B, D * bf, static_cast<uint64_t>(T) * D * bf,
-                   64, C::BM, CU_TENSOR_MAP_SWIZZLE_128B))
-        return SI_ERR_CUDA;
-    if (!encode_3d(&tw, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, w, H, S, B, H * 4ull, static_cast<uint64_t>(S) * H * 4ull,
-                   H, C::QT, CU_TENSOR_MAP_SWIZZLE_NONE))
-        return SI_ERR_CUDA;
-
-    uint32_t smem = C::dyn_bytes(smem_pool, p.P);
-    if (smem < kMinDynSmem) smem = kMinDynSmem;
-    if (smem + C::STATIC_BYTES > kMaxDynSmem) return SI_ERR_UNSUPPORTED;
-    auto kern = smem_pool ? si::select_kernel<H, D, true> : si::select_kernel<H, D, false>;
-    cudaFuncAttributes fa;
-    if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return SI_ERR_CUDA;
-    if (fa.sharedSizeBytes > C::STATIC_BYTES) return SI_ERR_UNSUPPORTED;  // build drifted past the bound
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    if (e != cudaSuccess) return cuda_fail("select kernel shared-memory attribute", e);
-    int64_t grid = sms < kMaxCtas ? sms : kMaxCtas;
-    if (grid > p.units) grid = p.units;
-    kern<<<static_cast<unsigned>(grid), C::THREADS, smem, stream>>>(tq, tkc, tw, p);
-    e = cudaGetLastError();
-    return e == cudaSuccess ? SI_OK : cuda_fail("select kernel launch", e);
-}
-
-// Query rows [t_lo, t_hi) of every batch; the whole problem is [0, S).
+// Query rows [t_lo, t_hi) of every batch; the whole problem is [0, S).  The
+// select kernel's instantiations live in one translation unit per H_I
+// (si_select_h*.cu); this picks the pools and the row sort and dispatches.
 si_status launch_select(const void* q, const float* w, const void* kc, int64_t B, int64_t S, int64_t T, int H, int D,
                         int m, int k, int32_t* out_idx, float* out_score, float* dense, void* ws,
                         cudaStream_t stream, int64_t t_lo = 0, int64_t t_hi = -1) {
-    if (t_hi < 0) t_hi = S;
-#define SI_CASE(HH, DD)     \
-    if (H == HH && D == DD) \
-        return launch_select_t<HH, DD>(q, w, kc, B, S, T, m, k, out_idx, out_score, dense, ws, stream, t_lo, t_hi);
-    SI_CASE(8, 64) SI_CASE(8, 128) SI_CASE(16, 64) SI_CASE(16, 128)
-    SI_CASE(32, 64) SI_CASE(32, 128) SI_CASE(64, 64) SI_CASE(64, 128)
-#undef SI_CASE
-    return SI_ERR_UNSUPPORTED;
+    si_host::SelectLaunch a{};
+    a.q = q;
+    a.w = w;
+    a.kc = kc;
+    a.B = B;
+    a.S = S;
+    a.T = T;
+    a.H = H;
+    a.D = D;
+    a.m = m;
+    a.k = dense ? 1 : k;
+    a.out_idx = out_idx;
+    a.out_score = out_score;
+    a.dense = dense;
+    a.ws = ws;
+    a.stream = stream;
+    a.t_lo = t_lo;
+    a.t_hi = t_hi < 0 ? S : t_hi;
+    const PoolPlan pp = dense ? PoolPlan{true, 0} : pool_plan(H, D, a.k);
+    a.smem_pool = pp.smem;
+    a.P = pp.P;
+    a.sort_e = (dense || !g_sort_in_select.load()) ? 0 : row_sort_e(H, D, k);
+    a.timeout_ns = g_timeout_ns.load();
+    a.gpool = pp.smem ? nullptr : reinterpret_cast<uint64_t*>(static_cast<uint8_t*>(ws) + kHeaderBytes);
+#ifdef SI_TRACE
+    // Tracing builds: per-warp cycle counters after the pools; the caller adds
+    // kMaxCtas * kTraceWarps * kTraceSlots * 8 bytes to the workspace.
+    a.trace = reinterpret_cast<unsigned long long*>(static_cast<uint8_t*>(ws) + kHeaderBytes +
+                                                    (pp.smem ? 0 : global_pool_bytes(H, D, a.k)));
+#endif
+    switch (H) {
+        case 8: return si_host::launch_select_h8(a);
+        case 16: return si_host::launch_select_h16(a);
+        case 32: return si_host::launch_select_h32(a);
+        case 64: return si_host::launch_select_h64(a);
+        default: return SI_ERR_UNSUPPORTED;
+    }
 }
+
+// Whether the select kernel leaves rows in their final order for these sizes.
+bool select_sorts_rows(int H, int D, int k) { return g_sort_in_select.load() && row_sort_e(H, D, k) > 0; }
 
 si_status launch_pad(int32_t* out_idx, float* out_score, int64_t n, cudaStream_t stream) {
     if (n <= 0) return SI_OK;
@@ -303,6 +300,7 @@ si_status si_indexer_topk(const void* q, const float* w, const void* kc, int64_t
     if (T == 0) return launch_pad(out_idx, out_score, B * S * k, s);
     st = launch_select(q, w, kc, B, S, T, H_I, d_I, m, k, out_idx, out_score, nullptr, workspace, s);
     if (st != SI_OK) return st;
+    if (select_sorts_rows(H_I, d_I, k)) return SI_OK;
     return si_sort_topk(out_idx, out_score, B * S, k, stream);
 }
 
@@ -326,6 +324,7 @@ si_status si_indexer_topk_rows(const void* q, const float* w, const void* kc, in
     }
     st = launch_select(q, w, kc, B, S, T, H_I, d_I, m, k, out_idx, out_score, nullptr, workspace, s, t_begin, t_end);
     if (st != SI_OK) return st;
+    if (select_sorts_rows(H_I, d_I, k)) return SI_OK;
     for (int64_t b = 0; b < B; ++b) {
         const int64_t off = (b * S + t_begin) * k;
         st = si_sort_topk(out_idx + off, out_score + off, n, k, stream);
@@ -378,6 +377,13 @@ si_status si_selftest_timeout(void* workspace, size_t workspace_bytes, uint64_t 
     si::timeout_selftest_kernel<<<1, 32, 0, s>>>(static_cast<uint32_t*>(workspace), limit_ns);
     return cudaGetLastError() == cudaSuccess ? SI_OK : SI_ERR_CUDA;
 }
+
+int si_select_sorts_rows(int H_I, int d_I, int k) {
+    if (!supported_h(H_I) || !supported_d(d_I) || k < 1 || k > 2048) return 0;
+    return select_sorts_rows(H_I, d_I, k) ? 1 : 0;
+}
+
+void si_set_sort_in_select(int enable) { g_sort_in_select.store(enable != 0); }
 
 void si_set_timeout_ns(uint64_t ns) {
     if (ns > 0) g_timeout_ns.store(ns);
@@ -460,7 +466,7 @@ extern "C" si_status si_indexer_topk_noalloc(const void* q, const float* w, cons
         st = launch_pad(out_idx, out_score, B * S * k, s);
     } else {
         st = launch_select(q, w, kc, B, S, T, H_I, d_I, m, k, out_idx, out_score, nullptr, ws, s);
-        if (st == SI_OK) st = si_sort_topk(out_idx, out_score, B * S, k, stream);
+        if (st == SI_OK && !select_sorts_rows(H_I, d_I, k)) st = si_sort_topk(out_idx, out_score, B * S, k, stream);
     }
     if (st != SI_OK) return st;
     if (out_status && cudaMemcpyAsync(out_status, ws, sizeof(uint32_t), cudaMemcpyDeviceToDevice, s) != cudaSuccess)

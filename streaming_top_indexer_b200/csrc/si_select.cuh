@@ -28,8 +28,9 @@
 // query's threshold (the current k-th best).  When a pool nears its capacity
 // P, one warp finds the k-th best pool entry by a most-significant-digit-first
 // radix select, keeps exactly the k best entries and raises the threshold.
-// At the end of a unit the pool is cut to k and written, unsorted, to the
-// outputs; a separate kernel sorts each row.
+// At the end of a unit the pool is cut to exactly its k best keys, which the
+// half sorts in shared memory and registers and writes in their final order
+// (a separate row sort remains for the few shapes whose sort does not fit).
 #pragma once
 #include <cuda.h>
 
@@ -83,6 +84,7 @@ struct SelectParams {
     float* dense;       // dense-score mode: [B,S,T] fp32, else nullptr
     uint64_t* gpool;    // pools in global memory (per CTA QT*P), or nullptr
     uint32_t* err;      // device error word
+    int sort_e;         // > 0: rows are written sorted, 128 * sort_e >= k keys per row; 0: unordered
     uint64_t timeout_ns;
     unsigned long long* trace;  // SI_TRACE builds only: [grid][kTraceWarps][kTraceSlots]
 };
@@ -426,7 +428,7 @@ __device__ __forceinline__ uint32_t half_count_ge(const Keys& keys, uint64_t L, 
 // by the 128 threads of the half.  8 bits per pass from the most significant
 // bit in which the keys differ, on a shared 256-bin histogram; every warp
 // scans the histogram itself, so all threads reach the same decision.
-__device__ __noinline__ uint64_t half_radix_bound(const uint64_t* pool, const PoolRegions& rg, int k, uint32_t slack,
+static __device__ __noinline__ uint64_t half_radix_bound(const uint64_t* pool, const PoolRegions& rg, int k, uint32_t slack,
                                                   CutScratch& cs, int tid, uint32_t bar_id) {
     const int lane = tid & 31, wq = tid >> 5;
     uint64_t kmin = ~0ull, kmax = 0ull;
@@ -778,7 +780,7 @@ __device__ __forceinline__ uint32_t half_walk_reg(const RegKeys& rk, uint64_t L,
 // 128 threads of the half.  Returns the new lower bound; `kept` gets the count.
 // `big`: the group's shared-memory candidate buffer (STREAM_CAND keys) when
 // the pools are in the workspace, else null.
-__device__ __noinline__ uint64_t cut_pool(uint64_t* pq, PoolRegions rg, int k, uint32_t max_keep, uint64_t lb,
+static __device__ __noinline__ uint64_t cut_pool(uint64_t* pq, PoolRegions rg, int k, uint32_t max_keep, uint64_t lb,
                                           CutScratch& cs, int tid, uint32_t bar_id, uint32_t& phase,
                                           uint32_t& kept, uint64_t* big, int big_cap) {
     uint64_t L = lb;
@@ -802,14 +804,108 @@ __device__ __noinline__ uint64_t cut_pool(uint64_t* pq, PoolRegions rg, int k, u
     return L;
 }
 
-// Writes the k best keys of one query's pool (or all, when fewer), unordered,
-// to its output row, then pads the row with (-1, -inf); by the half.  The
-// kept keys are packed first -- into the shared-memory buffer `big` when the
-// pool is in the workspace (k <= 2048 < STREAM_CAND), else to the front of
-// the shared-memory pool -- so that the row is written with coalesced stores.
-__device__ __noinline__ void emit_best(uint64_t* pq, PoolRegions rg, int k, CutScratch& cs, int tid,
+// Sorts the n packed keys buf[0, n) of one query (n <= k <= 128*E) in
+// descending key order -- score descending, then key index ascending -- and
+// writes the row's k entries, padding (-1, -inf) past n; by the 128 threads
+// of the half.  A bitonic network over 128*E keys: element i is slot i%E of
+// thread i/E (zero keys, below every real key, fill [n, 128*E)).  Partner
+// distances below E are register swaps, those below 32*E lane shuffles, and
+// the rest (the last three stages' worth) exchange through buf itself, which
+// must hold 128*E keys.  Each thread then writes E consecutive row entries.
+template <int E>
+__device__ __noinline__ void half_sort_emit(uint64_t* buf, int n, int k, int tid, uint32_t bar_id, int32_t* out_idx,
+                                            float* out_score) {
+    constexpr int K2 = 128 * E;
+    uint64_t v[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+        const int i = tid * E + e;
+        v[e] = i < n ? buf[i] : 0ull;
+    }
+    bar_sync(bar_id, 128);  // every key is in registers before buf serves the exchanges
+#pragma unroll
+    for (int size = 2; size <= K2; size <<= 1) {
+#pragma unroll
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            if (stride < E) {
+#pragma unroll
+                for (int e = 0; e < E; ++e) {
+                    const int pe = e ^ stride;
+                    if (pe > e) {
+                        // keys are distinct (zero fill keys are equal, and swapping
+                        // them changes nothing), so one compare decides
+                        const bool desc = ((tid * E + e) & size) == 0;
+                        const uint64_t a = v[e], b = v[pe];
+                        const bool sw = (a < b) == desc;
+                        v[e] = sw ? b : a;
+                        v[pe] = sw ? a : b;
+                    }
+                }
+            } else {
+                const int pt = stride / E;  // partner thread distance
+                const bool lower = (tid & pt) == 0;
+                uint64_t o[E];
+                if (stride < 32 * E) {
+#pragma unroll
+                    for (int e = 0; e < E; ++e) o[e] = __shfl_xor_sync(0xffffffffu, v[e], pt);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < E; ++e) buf[tid * E + e] = v[e];
+                    bar_sync(bar_id, 128);
+#pragma unroll
+                    for (int e = 0; e < E; ++e) o[e] = buf[(tid ^ pt) * E + e];
+                    bar_sync(bar_id, 128);  // read before the next exchange overwrites
+                }
+#pragma unroll
+                for (int e = 0; e < E; ++e) {
+                    const bool desc = ((tid * E + e) & size) == 0;
+                    const bool take_max = (lower == desc);
+                    v[e] = ((v[e] > o[e]) == take_max) ? v[e] : o[e];
+                }
+            }
+        }
+    }
+    const int i0 = tid * E;
+    if constexpr (E >= 4) {
+        const bool vec = ((reinterpret_cast<uintptr_t>(out_idx + i0) | reinterpret_cast<uintptr_t>(out_score + i0)) &
+                          15u) == 0 && i0 + E <= k;
+        if (vec) {
+#pragma unroll
+            for (int c = 0; c < E / 4; ++c) {
+                int32_t ix[4];
+                float sc[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const bool real = i0 + 4 * c + u < n;
+                    ix[u] = real ? key_index(v[4 * c + u]) : -1;
+                    sc[u] = real ? key_score(v[4 * c + u]) : -__int_as_float(0x7f800000);
+                }
+                reinterpret_cast<int4*>(out_idx + i0)[c] = make_int4(ix[0], ix[1], ix[2], ix[3]);
+                reinterpret_cast<float4*>(out_score + i0)[c] = make_float4(sc[0], sc[1], sc[2], sc[3]);
+            }
+            return;
+        }
+    }
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+        const int i = i0 + e;
+        if (i < k) {
+            const bool real = i < n;
+            out_idx[i] = real ? key_index(v[e]) : -1;
+            out_score[i] = real ? key_score(v[e]) : -__int_as_float(0x7f800000);
+        }
+    }
+}
+
+// Writes the k best keys of one query's pool (or all, when fewer) to its
+// output row, then pads the row with (-1, -inf); by the half.  The kept keys
+// are packed first -- into the shared-memory buffer `big` when the pool is in
+// the workspace (k <= 2048 < STREAM_CAND), else to the front of the shared-
+// memory pool.  With sort_e > 0 they are then sorted (half_sort_emit) and the
+// row is final; otherwise the row is written in pool order, unsorted.
+static __device__ __noinline__ void emit_best(uint64_t* pq, PoolRegions rg, int k, CutScratch& cs, int tid,
                                        uint32_t bar_id, uint32_t& phase, int32_t* out_idx, float* out_score,
-                                       uint64_t* big, int big_cap) {
+                                       uint64_t* big, int big_cap, int sort_e) {
     uint64_t* dst = big ? big : pq;
     auto pack = [&](uint64_t x, uint32_t pos) { dst[pos] = x; };
     const uint32_t ku = static_cast<uint32_t>(k);
@@ -833,6 +929,16 @@ __device__ __noinline__ void emit_best(uint64_t* pq, PoolRegions rg, int k, CutS
         out = half_walk_kept(pq, rg, L, cs, tid, bar_id, phase, pack);
     }
     bar_sync(bar_id, 128);  // the packed keys are visible to the whole half
+    // With sort_e set, the row is written in its final order; the packed keys'
+    // buffer (the pool, or `big`) holds at least 128 * sort_e keys.
+    switch (sort_e) {
+        case 1: half_sort_emit<1>(dst, static_cast<int>(out), k, tid, bar_id, out_idx, out_score); return;
+        case 2: half_sort_emit<2>(dst, static_cast<int>(out), k, tid, bar_id, out_idx, out_score); return;
+        case 4: half_sort_emit<4>(dst, static_cast<int>(out), k, tid, bar_id, out_idx, out_score); return;
+        case 8: half_sort_emit<8>(dst, static_cast<int>(out), k, tid, bar_id, out_idx, out_score); return;
+        case 16: half_sort_emit<16>(dst, static_cast<int>(out), k, tid, bar_id, out_idx, out_score); return;
+        default: break;
+    }
     for (int i = tid; i < k; i += 128) {
         if (i < static_cast<int>(out)) {
             const uint64_t x = dst[i];
@@ -1013,7 +1119,15 @@ __global__ void __launch_bounds__(SelCfg<H, D>::THREADS, 1)
                                   smem_desc_sw128(b_base + c * C::Q_CHUNK + off), idesc, kk > 0 ? 1u : 0u);
                     }
                     umma_commit(bar(kBarKcEmpty + st));
+#ifdef SI_FAULT_TEST
+                    // Test builds only (never the product library): CTA 0 does not
+                    // signal its third accumulator.  The epilogue's bounded wait on it
+                    // runs out, which exercises the abort path end to end: error word,
+                    // abort flag, drain of issued loads and MMAs, TMEM release.
+                    if (!(cta == 0 && acc_it == 2)) umma_commit(bar(kBarAccFull + buf));
+#else
                     umma_commit(bar(kBarAccFull + buf));
+#endif
                     issued = true;
                     ++kc_it;
                     ++acc_it;
@@ -1220,7 +1334,7 @@ __global__ void __launch_bounds__(SelCfg<H, D>::THREADS, 1)
                     if (t >= p.t_hi) continue;  // uniform over the half
                     const int64_t row = (ui.b * p.S + t) * static_cast<int64_t>(k);
                     emit_best(pool + qi * P, pool_regions(kp[q], fw(q), cntw[half][q]), k, cs, htid, bar_id, cphase,
-                              p.out_idx + row, p.out_score + row, big, C::STREAM_CAND);
+                              p.out_idx + row, p.out_score + row, big, C::STREAM_CAND, p.sort_e);
                     bar_sync(bar_id, 128);
                 }
             }

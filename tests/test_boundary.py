@@ -127,3 +127,15 @@ def test_host_row_windows():
         for a, b in win:
             assert a < b and a % 256 == 0 and (b % 256 == 0 or b == S)
         assert len(win) <= max(1, chunks) + 1
+
+
+def test_select_sorts_rows_host_arithmetic(lib):
+    """The select kernel sorts rows in place for k <= 1024 (128*E >= k keys,
+    E <= 8 a power of two); larger k keeps the separate row sort."""
+    for H, D in [(64, 128), (64, 64), (32, 128), (32, 64), (16, 128), (16, 64), (8, 128), (8, 64)]:
+        for k in (1, 64, 128, 129, 512, 600, 1024):
+            assert si.select_sorts_rows(H, D, k), (H, D, k)
+        for k in (1025, 1089, 2048):  # 16 keys per thread: the separate row sort is faster
+            assert not si.select_sorts_rows(H, D, k), (H, D, k)
+    assert not si.select_sorts_rows(64, 128, 0) and not si.select_sorts_rows(64, 128, 2049)
+    assert not si.select_sorts_rows(48, 128, 64)

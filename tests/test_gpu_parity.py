@@ -115,13 +115,47 @@ def test_deterministic_repeat():
     assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
 
 
-def test_select_then_sort_equals_indexer_topk():
+def test_select_output_is_already_sorted():
+    """The select kernel sorts each row at unit end: its output alone equals
+    the full call, and sorting it again changes nothing."""
     q, w, kc = make(1, 3000, 750, 64, 128, 4, 128, seed=13)
+    assert si.select_sorts_rows(64, 128, 128)
     idx, sc = gh.gpu_topk(q, w, kc, 4, 128)
     i2, s2 = si.select_topk(q, w, kc, 4, 128)
+    torch.cuda.synchronize()
+    assert torch.equal(idx, i2) and torch.equal(sc, s2)
     si.sort_topk(i2, s2)
     torch.cuda.synchronize()
     assert torch.equal(idx, i2) and torch.equal(sc, s2)
+
+
+SORT_CASES = [
+    # B, S, T, H, D, m, k   (keys per thread of the unit-end sort, pools)
+    (1, 1000, 250, 64, 128, 4, 100),    # E=1, shared-memory pools
+    (2, 777, 300, 32, 128, 2, 200),     # E=2
+    (1, 2000, 500, 64, 64, 4, 600),     # E=8 with k > T (padding inside the sorted rows)
+    (1, 9000, 2250, 64, 128, 4, 512),   # E=4, several cuts per query
+    (1, 5000, 1250, 64, 128, 4, 1024),  # E=8, shared-memory pools of 1856
+    (1, 3000, 750, 64, 128, 4, 1050),   # k > 1024: the kernel leaves rows unordered, the row sort runs
+    (1, 2000, 500, 32, 128, 4, 700),    # E=8, workspace pools (the shared-memory buffer)
+    (2, 1100, 275, 16, 128, 4, 300),    # H=16: workspace pools, E=4
+    (3, 160, 20, 8, 128, 7, 5),         # H=8: 16 queries per half
+]
+
+
+@pytest.mark.parametrize("B,S,T,H,D,m,k", SORT_CASES)
+def test_in_kernel_sort_equals_separate_sort(B, S, T, H, D, m, k):
+    """Rows sorted at unit end inside the select kernel are bit-identical to
+    unordered rows sorted by the separate row-sort kernel."""
+    q, w, kc = make(B, S, T, H, D, m, k, seed=B * 77 + S + k)
+    a_idx, a_sc = gh.gpu_topk(q, w, kc, m, k)
+    si.set_sort_in_select(False)
+    try:
+        b_idx, b_sc = gh.gpu_topk(q, w, kc, m, k)
+    finally:
+        si.set_sort_in_select(True)
+    assert torch.equal(a_idx, b_idx)
+    assert torch.equal(a_sc.view(torch.int32), b_sc.view(torch.int32))
 
 
 def test_zero_keys_gives_padding():
