@@ -371,6 +371,10 @@ def run_ours(args, world, rank, local):
             "workspace_bytes": ws_bytes, "gpu_launches": launches_per_step * args.steps, "roofline": roofline,
             "clocks": sampler.summary()}
 
+    if args.csa:
+        att = attention_measure(si, idx, wl, args, dev, stream, peaks, peak_src)
+        att["indexer_plus_attention_ms"] = ms_per_step + att["ms"]
+        line["csa_attention"] = att
     # end to end through the public API with host buffers
     if not args.no_e2e:
         line["e2e"] = e2e_measure(si, q, w, kc, wl, args, world, dev, stream, flops_rank)
@@ -472,6 +476,50 @@ def run_sweep(args):
         del idx, sc, ws
 
 
+def attention_pairs(S: int, T: int, m: int, k: int) -> int:
+    """Number of (query row, selected key) pairs: sum_t min(k, V_t)."""
+    t = np.arange(S, dtype=np.int64)
+    return int(np.minimum(k, np.minimum(T, (t + 1) // m)).sum())
+
+
+def attention_measure(si, idx, wl, args, dev, stream, peaks, peak_src):
+    """The CSA step's third stage on the indexer's output: sparse attention of
+    128 heads (d = d_v = 128, bf16) over the selected keys, CUDA-event timed
+    on the same stream.  FLOPs: 2*128*(d + d_v) per (row, selected key)."""
+    from streaming_top_indexer_b200 import synth
+    D = DV = 128
+    q, kc, vc = synth.generate_attention(wl.B, wl.S, wl.T, D, DV, seed=args.seed, device=dev)
+    out = torch.empty((wl.B, wl.S, 128, DV), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((wl.B, wl.S, 128), dtype=torch.float32, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    scale = 1.0 / math.sqrt(D)
+    for _ in range(args.warmup):
+        si.sparse_attention(q, kc, vc, idx, scale, out, lse, status, stream)
+    torch.cuda.synchronize(dev)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for e0, e1 in ev:
+        e0.record(stream)
+        si.sparse_attention(q, kc, vc, idx, scale, out, lse, status, stream)
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    assert int(status.item()) == 0, "device error in the attention stage"
+    ms = statistics.mean(e0.elapsed_time(e1) for e0, e1 in ev)
+    pairs = wl.B * attention_pairs(wl.S, wl.T, wl.m, wl.k)
+    flops = 2.0 * 128 * (D + DV) * pairs
+    tflops = flops / (ms * 1e-3) / 1e12
+    # bytes: q and out once, the gathered K and V rows (from L2 when they fit)
+    hbm = q.numel() * 2 + out.numel() * 2 + lse.numel() * 4 + idx.numel() * 4
+    gathered = pairs * (D + DV) * 2
+    del q, kc, vc, out, lse
+    return {"kernel": "sparse_attn_kernel<128,128>", "heads": 128, "d": D, "d_v": DV, "ms": ms,
+            "value": tflops, "unit": "TFLOP/s",
+            "roofline": {"bound": "tensor", "achieved": tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": tflops / peaks["bf16_tflops"], "peak_source": f"{peak_src} bf16 burst"},
+            "hbm_bytes_per_call": int(hbm), "hbm_gbs": hbm / (ms * 1e-3) / 1e9,
+            "gathered_kv_bytes_per_call": int(gathered),
+            "indexer_plus_attention_ms": None}
+
+
 def e2e_measure(si, q, w, kc, wl, args, world, dev, stream, flops_rank):
     """Same metric through indexer_topk_host: pinned host inputs copied in,
     outputs copied out, inside the timed region every step."""
@@ -510,6 +558,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--csa", action="store_true",
+                    help="also time CSA's sparse attention (128 heads, d=d_v=128) over the indexer's output")
     ap.add_argument("--sort-kernel", action="store_true",
                     help="sort rows in the separate row-sort kernel instead of inside the select kernel")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work")

@@ -194,6 +194,33 @@ SI_API int si_select_sorts_rows(int H_I, int d_I, int k);
  * identical results; the switch exists to time the two designs. */
 SI_API void si_set_sort_in_select(int enable);
 
+/* The sparse attention stage of CSA, over the keys the indexer selected
+ * (StreamIndex: Memory-Bounded Compressed Sparse Attention via Streaming
+ * Top-k, Abstract: the attention reads only the selected compressed keys; the
+ * Abstract gives no formula, and this is the plainest reading):
+ *
+ *     out[b,t,h,:] = sum_j softmax_j(scale * q[b,t,h,:] . K[b,j,:]) V[b,j,:]
+ *     lse[b,t,h]   = log sum_j exp(scale * q[b,t,h,:] . K[b,j,:])
+ *
+ * with j over the entries idx[b,t,0..k) in [0, T); other entries (the
+ * indexer's -1 padding) are skipped.  A row with no such entry gives
+ * out = 0 and lse = -infinity.  K and V are shared by all heads.
+ *   q:      bf16 [B,S,H_a,d]   (H_a = 128: one head per MMA row)
+ *   kcache: bf16 [B,T,d]       compressed keys;  vcache: bf16 [B,T,d_v]
+ *   idx:    int32 [B,S,k]      e.g. si_indexer_topk's out_idx
+ *   out:    bf16 [B,S,H_a,d_v];  lse: fp32 [B,S,H_a]
+ *   status: a device word, set to 0 by the call and to SI_ERR_TIMEOUT if a
+ *           bounded device wait expired (read it after the stream reaches
+ *           the end of the call).
+ * Supported: H_a = 128; d, d_v in {64, 128}; 1 <= k <= 2048;
+ * B*S*128 < 2^31; B*T < 2^31.  q, kcache, vcache and out 16-byte aligned;
+ * idx, lse and status 4-byte aligned.  Allocates nothing; asynchronous on
+ * `stream`.  Arithmetic: bf16 products, fp32 accumulation, softmax weights
+ * rounded to bf16 for the P.V product (sums in fp32), bf16 output. */
+SI_API si_status si_sparse_attention(const void* q, const void* kcache, const void* vcache, const int32_t* idx,
+                                     int64_t B, int64_t S, int64_t T, int H_a, int d, int d_v, int k,
+                                     float scale, void* out, float* lse, uint32_t* status, si_stream_t stream);
+
 /* Device-side wait limit, in nanoseconds, used by later calls (default 2 s). */
 SI_API void si_set_timeout_ns(uint64_t ns);
 

@@ -23,7 +23,7 @@ __all__ = [
     "SIError", "library_path", "load_library", "workspace_bytes", "indexer_topk",
     "select_topk", "sort_topk", "indexer_scores", "check_device_status",
     "selftest_timeout", "set_timeout_ns", "indexer_topk_host", "version", "select_sorts_rows",
-    "set_sort_in_select",
+    "set_sort_in_select", "sparse_attention",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -68,6 +68,9 @@ def _declare(lib):
     lib.si_selftest_timeout.argtypes = [vp, sz, c.c_uint64, vp]
     lib.si_set_timeout_ns.restype = None
     lib.si_set_timeout_ns.argtypes = [c.c_uint64]
+    lib.si_sparse_attention.restype = c.c_int
+    lib.si_sparse_attention.argtypes = [vp, vp, vp, vp, i64, i64, i64, i32, i32, i32, i32, c.c_float, vp, vp, vp,
+                                        vp]
     lib.si_select_sorts_rows.restype = c.c_int
     lib.si_select_sorts_rows.argtypes = [i32, i32, i32]
     lib.si_set_sort_in_select.restype = None
@@ -326,3 +329,34 @@ def indexer_topk_host(q, w, kc, m: int, k: int, device="cuda", buffers=None, str
             b["score_h"][:, t0:t1].copy_(b["score"][:, t0:t1], non_blocking=True)
     s.wait_stream(s_out)
     return b["idx_h"], b["score_h"]
+
+def sparse_attention(q, kcache, vcache, idx, scale: float, out=None, lse=None, status=None, stream=None):
+    """CSA sparse attention over the selected keys (si_sparse_attention).
+
+    q bf16 [B,S,128,d], kcache bf16 [B,T,d], vcache bf16 [B,T,d_v], idx int32
+    [B,S,k] (entries outside [0,T) are skipped).  Returns (out bf16
+    [B,S,128,d_v], lse fp32 [B,S,128], status int32 [1] device word: 0, or 6
+    if a device wait expired), asynchronously on ``stream``.
+    """
+    _need(q, "q", torch.bfloat16, 4)
+    _need(kcache, "kcache", torch.bfloat16, 3)
+    _need(vcache, "vcache", torch.bfloat16, 3)
+    _need(idx, "idx", torch.int32, 3)
+    B, S, H, D = q.shape
+    T, DV = kcache.shape[1], vcache.shape[2]
+    k = idx.shape[2]
+    if kcache.shape[0] != B or vcache.shape[:2] != (B, T) or kcache.shape[2] != D or tuple(idx.shape[:2]) != (B, S):
+        raise ValueError("shape mismatch")
+    if out is None:
+        out = torch.empty((B, S, H, DV), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, S, H), dtype=torch.float32, device=q.device)
+    if status is None:
+        status = torch.empty(1, dtype=torch.int32, device=q.device)
+    _need(out, "out", torch.bfloat16, 4)
+    _need(lse, "lse", torch.float32, 3)
+    _check(load_library().si_sparse_attention(q.data_ptr(), kcache.data_ptr() if T > 0 else None,
+                                              vcache.data_ptr() if T > 0 else None, idx.data_ptr(), B, S, T, H, D,
+                                              DV, k, float(scale), out.data_ptr(), lse.data_ptr(),
+                                              status.data_ptr(), _stream(stream)), "si_sparse_attention")
+    return out, lse, status

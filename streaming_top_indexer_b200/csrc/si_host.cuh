@@ -44,6 +44,9 @@ struct SelectLaunch {
 // Defined in si_lib.cu.
 si_status cuda_fail(const char* where, cudaError_t e);
 int device_sms(int dev);
+uint64_t timeout_ns();  // device wait limit set by si_set_timeout_ns
+bool encode_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t d0, uint64_t d1,
+               uint64_t stride1_bytes, uint32_t box0, uint32_t box1, CUtensorMapSwizzle sw);
 bool encode_3d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
                uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t box0, uint32_t box1, CUtensorMapSwizzle sw);
 

@@ -58,6 +58,20 @@ bool encode_3d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint6
     return r == CUDA_SUCCESS;
 }
 
+bool encode_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t d0, uint64_t d1,
+               uint64_t stride1_bytes, uint32_t box0, uint32_t box1, CUtensorMapSwizzle sw) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {d0, d1};
+    cuuint64_t strides[1] = {stride1_bytes};
+    cuuint32_t box[2] = {box0, box1};
+    cuuint32_t estr[2] = {1, 1};
+    std::memset(map, 0, sizeof(*map));
+    CUresult r = enc(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 namespace {
 std::mutex g_dev_mu;
 int g_dev_sms[64] = {};
@@ -77,6 +91,12 @@ int device_sms(int dev) {
 }  // namespace si_host
 
 namespace {
+std::atomic<uint64_t> g_timeout_ns{2000000000ull};
+}  // namespace
+
+uint64_t si_host::timeout_ns() { return g_timeout_ns.load(); }
+
+namespace {
 
 using si_host::cuda_fail;
 using si_host::kHeaderBytes;
@@ -85,7 +105,6 @@ using si_host::kMaxDynSmem;
 // Row windows of si_indexer_topk_rows start (and, except at S, end) on
 // multiples of this, a multiple of every unit's query count (256/H_I).
 constexpr int64_t kRowAlign = 256;
-std::atomic<uint64_t> g_timeout_ns{2000000000ull};
 // Whether the select kernel sorts each row at unit end (default) or leaves the
 // rows unordered for the separate row sort.
 std::atomic<bool> g_sort_in_select{true};

@@ -152,3 +152,24 @@ def checked_rows(S: int, m: int, k: int, b: int, seed: int = 0, n: int = 512):
 def bf16_bits(t: torch.Tensor) -> np.ndarray:
     """Raw bf16 bit patterns of a tensor as a host uint16 array."""
     return t.detach().contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+ATTN_HEADS = 128
+
+
+def generate_attention(B: int, S: int, T: int, D: int = 128, DV: int = 128, seed: int = 0, device="cpu"):
+    """Draw the sparse attention's inputs: q bf16 [B,S,128,D], kcache bf16
+    [B,T,D] and vcache bf16 [B,T,DV], N(0,1) values rounded to bf16 (q drawn
+    in fixed row blocks like generate), from one seeded generator."""
+    dev = torch.device(device)
+    g = torch.Generator(device=dev)
+    g.manual_seed(seed + 7777)
+    q = torch.empty((B, S, ATTN_HEADS, D), dtype=torch.bfloat16, device=dev)
+    rows = max(1, Q_BLOCK_ELEMS // (ATTN_HEADS * D))
+    for b in range(B):
+        for s0 in range(0, S, rows):
+            s1 = min(S, s0 + rows)
+            q[b, s0:s1].copy_(torch.randn((s1 - s0, ATTN_HEADS, D), generator=g, device=dev, dtype=torch.float32))
+    kc = torch.randn((B, T, D), generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+    vc = torch.randn((B, T, DV), generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+    return q, kc, vc

@@ -143,3 +143,40 @@ def check_rows(g_idx, g_score, o_idx, o_score, o_meta, o_scores, k, bound, where
     assert rep["recall_mean"] >= RECALL_MEAN, f"{where}: mean recall {rep['recall_mean']}"
     assert rep["recall_min"] >= RECALL_MIN, f"{where}: min recall {rep['recall_min']}"
     return rep
+
+
+def attention_tolerance(q_rows_bits, kc_bits, row_b, idx_rows, scale, absw, ref_out, ref_lse):
+    """First-order error bounds of the GPU sparse attention against the fp64
+    oracle, per output element and per lse value.
+
+    The kernel computes each score in fp32 from exact bf16 products
+    (error e_j <= d * 2^-23 * scale * sum_d |q_d K_jd|), exponentiates with
+    ex2.approx (relative error below 2^-21), rounds the weights to bf16 for
+    the P.V product while l sums them in fp32, accumulates in fp32
+    (n * 2^-23 relative of sum_j p_j |V_j|), and rounds the output to bf16.
+    bf16 keeps 8 significant bits, so each of its roundings is within 2^-8
+    relative.  With E = 2 * max_j e_j over the row's keys, n the number of
+    keys, A = sum_j p_j |V_j| (absw) and O the exact output:
+
+        |out - O| <= 1.1 * (2^-8 + E + n 2^-23 + 2^-20) * (A + |O|)
+        |lse - L| <= 1.1 * (E + n 2^-23 + 2^-19) + 2^-22 |L|
+    Returns (tol_out [R,H,DV], tol_lse [R,H])."""
+    def f64(bits):
+        return (np.asarray(bits, np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+    qa = np.abs(f64(q_rows_bits))                       # [R,H,D]
+    R, H, D = qa.shape
+    tol_out = np.zeros(ref_out.shape)
+    tol_lse = np.zeros(ref_lse.shape)
+    T = kc_bits.shape[1]
+    for r in range(R):
+        sel = idx_rows[r][(idx_rows[r] >= 0) & (idx_rows[r] < T)]
+        n = len(sel)
+        if n == 0:
+            continue
+        ka = np.abs(f64(kc_bits[row_b[r], sel]))        # [n, D]
+        E = 2 * D * FP32_ULP * abs(scale) * (qa[r] @ ka.T).max(axis=1)   # [H]
+        eps = 2.0 ** -8 + E + n * FP32_ULP + 2.0 ** -20
+        tol_out[r] = 1.1 * eps[:, None] * (absw[r] + np.abs(ref_out[r]))
+        tol_lse[r] = 1.1 * (E + n * FP32_ULP + 2.0 ** -19) + 2.0 ** -22 * np.abs(ref_lse[r])
+    return tol_out, tol_lse

@@ -94,3 +94,41 @@ def test_planted_mistakes_are_rejected(mistake):
     bound = checker.score_error_bound(q, w, kc, rb, g_idx)
     with pytest.raises(AssertionError):
         checker.check_rows(g_idx, g_sc, o_idx, o_sc, meta, scores, k, bound, mistake)
+
+
+def test_attention_bound_covers_kernel_arithmetic():
+    """The attention tolerance covers the kernel's arithmetic simulated on the
+    CPU: fp32 scores, base-2 softmax with bf16 weights for P.V and an fp32
+    sum l, fp32 accumulation, bf16 output.  Rows with few keys (where one
+    weight's bf16 rounding dominates) included."""
+    import torch
+    from oracle import attention as att
+    rng = np.random.default_rng(21)
+    B, T, H, D, DV = 1, 300, 16, 64, 32
+    q = pins.random_bf16(rng, (40, H, D))
+    K = pins.random_bf16(rng, (B, T, D))
+    V = pins.random_bf16(rng, (B, T, DV))
+    scale = 1 / np.sqrt(D)
+    idx = np.full((40, 64), -1, np.int32)
+    for r in range(40):
+        n = 1 + r if r < 30 else 64
+        idx[r, :n] = rng.choice(T, n, replace=False)
+    rb = np.zeros(40, np.int64)
+    ref, lse, absw = att.sparse_attention_rows(q, idx, rb, K, V, scale, want_absw=True)
+    tol, tol_lse = checker.attention_tolerance(q, K, rb, idx, scale, absw, ref, lse)
+    qf, kf, vf = _bits_to_f32(q), _bits_to_f32(K[0]), _bits_to_f32(V[0])
+    c2 = np.float32(scale * np.log2(np.e))
+    worst = 0.0
+    for r in range(40):
+        sel = idx[r][idx[r] >= 0]
+        s = (qf[r].astype(np.float32) @ kf[sel].T.astype(np.float32)).astype(np.float32)   # [H, n]
+        x = (s * c2).astype(np.float32)
+        p = np.exp2(x - x.max(axis=1, keepdims=True)).astype(np.float32)
+        l = p.sum(axis=1, dtype=np.float32)
+        pb = torch.from_numpy(p).to(torch.bfloat16).float().numpy()
+        o = (pb @ vf[sel]).astype(np.float32) / l[:, None]
+        ob = torch.from_numpy(o.astype(np.float32)).to(torch.bfloat16).double().numpy()
+        err = np.abs(ob - ref[r])
+        assert np.all(err <= tol[r]), (r, float((err / tol[r]).max()))
+        worst = max(worst, float((err / tol[r]).max()))
+    assert worst > 0.05  # the bound is not vacuous
