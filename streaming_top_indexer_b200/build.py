@@ -21,6 +21,8 @@ TRACE_LIB_PATH = os.path.join(LIB_DIR, "libsi_trace.so")  # cycle-tracing build 
 # Test-only build (SI_FAULT_TEST) whose select kernel withholds one signal so
 # that a bounded device wait expires; used by the abort-path GPU test only.
 FAULT_TEST_LIB_PATH = os.path.join(LIB_DIR, "libsi_ftest.so")
+# Timeline-tracing variant of the sparse attention kernel (SI_ATTN_TRACE).
+ATTN_TRACE_LIB_PATH = os.path.join(LIB_DIR, "libsi_atrace.so")
 # The host library, one translation unit per H_I of the select kernel and the
 # sparse attention stage, compiled in parallel and linked into one library.
 SOURCES = [os.path.join(CSRC, f) for f in ("si_lib.cu", "si_select_h8.cu", "si_select_h16.cu", "si_select_h32.cu",
@@ -103,7 +105,9 @@ def build(force: bool = False, verbose: bool = False, extra=(), trace: bool = Fa
 
 
 if __name__ == "__main__":
-    if "--fault-test" in sys.argv:
+    if "--attn-trace" in sys.argv:
+        print(build(verbose=True, extra=["-DSI_ATTN_TRACE"], out=ATTN_TRACE_LIB_PATH))
+    elif "--fault-test" in sys.argv:
         print(build_fault_test(force=True, verbose=True))
     else:
         print(build(force="--force" in sys.argv, verbose=True, trace="--trace" in sys.argv,

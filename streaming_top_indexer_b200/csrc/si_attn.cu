@@ -10,6 +10,14 @@
 #include "si_attn.cuh"
 #include "si_host.cuh"
 
+#ifdef SI_ATTN_TRACE
+// Tracing builds only: the timeline buffer and a reader for it.
+static __device__ unsigned long long g_attn_trace[4 * si::kATraceItems * 4];
+extern "C" __attribute__((visibility("default"))) int si_attn_trace_read(unsigned long long* host_out) {
+    return cudaMemcpyFromSymbol(host_out, g_attn_trace, sizeof(g_attn_trace)) == cudaSuccess ? 0 : 1;
+}
+#endif
+
 namespace {
 
 template <int D, int DV>
@@ -28,24 +36,21 @@ si_status launch_attn_t(const void* q, const void* kcache, const void* vcache, c
     p.k = k;
     p.nchunks = (k + C::NK - 1) / C::NK;
     p.idx = idx;
+    p.kcache = static_cast<const uint16_t*>(kcache);
+    p.vcache = static_cast<const uint16_t*>(vcache);
     p.out = static_cast<uint16_t*>(out);
     p.lse = lse;
     p.c2 = scale * 1.4426950408889634f;
     p.err = status;
     p.timeout_ns = si_host::timeout_ns();
+#ifdef SI_ATTN_TRACE
+    if (cudaGetSymbolAddress(reinterpret_cast<void**>(&p.trace), g_attn_trace) != cudaSuccess) return SI_ERR_CUDA;
+#endif
 
-    CUtensorMap tq, tk, tv;
+    CUtensorMap tq;
     const uint64_t rows = static_cast<uint64_t>(B * S);
-    const uint64_t keys = static_cast<uint64_t>(B * T);
     // q as [B*S*128 rows, d]: one row's heads are one 128-row box per 64 columns
     if (!si_host::encode_2d(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q, D, rows * C::HA, D * 2ull, 64, C::HA,
-                            CU_TENSOR_MAP_SWIZZLE_128B))
-        return SI_ERR_CUDA;
-    // the key / value caches as [B*T rows, d]: boxes one row high, for gather4
-    if (!si_host::encode_2d(&tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kcache, D, keys, D * 2ull, 64, 1,
-                            CU_TENSOR_MAP_SWIZZLE_128B))
-        return SI_ERR_CUDA;
-    if (!si_host::encode_2d(&tv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, vcache, DV, keys, DV * 2ull, 64, 1,
                             CU_TENSOR_MAP_SWIZZLE_128B))
         return SI_ERR_CUDA;
 
@@ -55,7 +60,7 @@ si_status launch_attn_t(const void* q, const void* kcache, const void* vcache, c
     if (e != cudaSuccess) return si_host::cuda_fail("attention kernel shared-memory attribute", e);
     int64_t grid = sms < si_host::kMaxCtas ? sms : si_host::kMaxCtas;
     if (grid > p.rows) grid = p.rows;
-    kern<<<static_cast<unsigned>(grid), C::THREADS, smem, stream>>>(tq, tk, tv, p);
+    kern<<<static_cast<unsigned>(grid), C::THREADS, smem, stream>>>(tq, p);
     e = cudaGetLastError();
     return e == cudaSuccess ? SI_OK : si_host::cuda_fail("attention kernel launch", e);
 }
