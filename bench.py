@@ -281,6 +281,12 @@ def run_ours(args, world, rank, local):
     dev = torch.device(f"cuda:{local}")
     wl = synth.WORKLOADS[args.workload]
     B, S, T, H, D, m, k = wl.B, wl.S, wl.T, wl.H, wl.D, wl.m, wl.k
+    # The per-head materialise baseline needs 4*B*S*H_I*(S/m) bytes for its fp32
+    # score tensor (Abstract): the largest S that fits this device's free memory.
+    free_start = torch.cuda.mem_get_info(dev)[0]
+    materialise = {"bytes_at_workload": 4 * B * S * H * T, "free_bytes": int(free_start),
+                   "s_max_fitting": int((free_start / (4 * B * H / m)) ** 0.5),
+                   "fits_at_workload": 4 * B * S * H * T <= free_start}
     q, w, kc = synth.generate(wl, seed=args.seed + rank, device=dev)
     # Peak HBM of the indexer step: counted from here, with the inputs resident
     # (generation's own temporaries are freed and not counted).
@@ -368,6 +374,7 @@ def run_ours(args, world, rank, local):
                                     "workspace": int(ws_bytes),
                                     "outputs_workspace_mem_get_info": int(mem_get_info_bytes)},
             "peak_hbm_scope": "allocator peak during the indexer calls, inputs resident, input generation excluded",
+            "materialise_baseline": materialise,
             "workspace_bytes": ws_bytes, "gpu_launches": launches_per_step * args.steps, "roofline": roofline,
             "clocks": sampler.summary()}
 
@@ -411,15 +418,22 @@ def run_sweep(args):
         sbuild.build()
     dev = torch.device("cuda:0")
     base = synth.WORKLOADS[args.workload]
+    # cells: (S, k, tuning); tuning = si_set_tuning's design parameters (the
+    # counterparts of the pages' chunk and key-tile sizes), defaults elsewhere
+    vals = [int(v) for v in args.sweep_values.split(",")] if args.sweep_values else None
     if args.sweep == "k":
-        cells = [(base.S, int(v)) for v in args.sweep_values.split(",")] if args.sweep_values else \
-            [(base.S, v) for v in (64, 128, 256, 512, 1024, 2048)]
+        cells = [(base.S, v, {}) for v in (vals or (64, 128, 256, 512, 1024, 2048))]
+    elif args.sweep == "s":
+        cells = [(v, base.k, {}) for v in (vals or (16384, 32768, 65536, 131072, 262144))]
     else:
-        cells = [(int(v), base.k) for v in args.sweep_values.split(",")] if args.sweep_values else \
-            [(v, base.k) for v in (16384, 32768, 65536, 131072, 262144)]
+        key = {"pool": "pool_entries", "check": "check_tiles", "slack": "cut_slack"}[args.sweep]
+        default = {"pool": (800, 1056, 1344, 1600, 1856), "check": (1, 2, 3, 4, 6),
+                   "slack": (32, 64, 128, 256, 512)}[args.sweep]
+        cells = [(base.S, base.k, {key: v}) for v in (vals or default)]
     stream = torch.cuda.current_stream(dev)
     dense_cache = {}
-    for S, k in cells:
+    for S, k, tuning in cells:
+        si.set_tuning(**tuning)
         wl = synth.Workload(f"{base.name}-sweep", base.B, S, base.m, base.H, base.D, k, base.kind)
         B, T, H, D, m = wl.B, wl.T, wl.H, wl.D, wl.m
         if S not in dense_cache:
@@ -453,7 +467,7 @@ def run_sweep(args):
         peak_idx = inputs + torch.cuda.max_memory_allocated(dev) - base_bytes
         cell = {"sweep": args.sweep, "workload": base.name, "B": B, "S": S, "T": T, "H_I": H, "d_I": D, "m": m,
                 "k": k, "value": flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms": ms,
-                "steps": args.steps, "warmup": args.warmup, "peak_hbm_bytes": int(peak_idx),
+                "tuning": tuning, "steps": args.steps, "warmup": args.warmup, "peak_hbm_bytes": int(peak_idx),
                 "recall_vs_materialised": None}
         if dense is not None:
             g = torch.Generator().manual_seed(args.seed + 1)
@@ -474,6 +488,7 @@ def run_sweep(args):
                                               "rows_identical": exact}
         print(json.dumps(cell), flush=True)
         del idx, sc, ws
+    si.set_tuning()
 
 
 def attention_pairs(S: int, T: int, m: int, k: int) -> int:
@@ -564,8 +579,9 @@ def main():
                     help="sort rows in the separate row-sort kernel instead of inside the select kernel")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work")
     ap.add_argument("--ref-budget", type=float, default=60.0, help="seconds of oracle work, reference arm")
-    ap.add_argument("--sweep", choices=["k", "s"], default=None,
-                    help="design-space sweep over k or S (one GPU; one JSON line per cell)")
+    ap.add_argument("--sweep", choices=["k", "s", "pool", "check", "slack"], default=None,
+                    help="design-space sweep over k, S, pool capacity, check interval or cut slack "
+                         "(one GPU; one JSON line per cell)")
     ap.add_argument("--sweep-values", default="", help="comma-separated k or S values of the sweep")
     ap.add_argument("--sweep-rows", type=int, default=256, help="rows checked against the materialised top-k")
     ap.add_argument("--sweep-dense-bytes", type=float, default=20e9,

@@ -221,6 +221,24 @@ SI_API si_status si_sparse_attention(const void* q, const void* kcache, const vo
                                      int64_t B, int64_t S, int64_t T, int H_a, int d, int d_v, int k,
                                      float scale, void* out, float* lse, uint32_t* status, si_stream_t stream);
 
+/* Design parameters of the select kernel, process-wide, for later calls and
+ * si_workspace_bytes (0 keeps a default).  They are the counterparts of the
+ * driver parameters the pages sweep (StreamIndex: Memory-Bounded Compressed
+ * Sparse Attention via Streaming Top-k, Abstract: chunk size, key-tile size):
+ *   pool_entries  candidates a query's pool holds between partition-merges
+ *                 (default: as many as shared memory allows, at least
+ *                 max(k+288, min(2k, k+768)); else 4k in the workspace).  It
+ *                 is raised to k + 4*(32*check_tiles+1) + 28 if smaller.  It
+ *                 stays in shared memory when it fits, else goes to the workspace;
+ *   cut_slack     entries above k an intermediate merge may keep (default 256);
+ *   check_tiles   128-key tiles streamed between two checks of the pools'
+ *                 fill (default 2).
+ * Results do not depend on them: every setting returns the exact top-k.
+ * Returns SI_ERR_INVALID_ARG (and changes nothing) for pool_entries outside
+ * [0, 65504], cut_slack outside [0, 4096] or check_tiles outside [0, 16].
+ * The workspace size depends on pool_entries: size it after the call. */
+SI_API si_status si_set_tuning(int pool_entries, int cut_slack, int check_tiles);
+
 /* Device-side wait limit, in nanoseconds, used by later calls (default 2 s). */
 SI_API void si_set_timeout_ns(uint64_t ns);
 

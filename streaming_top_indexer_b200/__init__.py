@@ -23,7 +23,7 @@ __all__ = [
     "SIError", "library_path", "load_library", "workspace_bytes", "indexer_topk",
     "select_topk", "sort_topk", "indexer_scores", "check_device_status",
     "selftest_timeout", "set_timeout_ns", "indexer_topk_host", "version", "select_sorts_rows",
-    "set_sort_in_select", "sparse_attention",
+    "set_sort_in_select", "sparse_attention", "set_tuning",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -75,6 +75,8 @@ def _declare(lib):
     lib.si_select_sorts_rows.argtypes = [i32, i32, i32]
     lib.si_set_sort_in_select.restype = None
     lib.si_set_sort_in_select.argtypes = [i32]
+    lib.si_set_tuning.restype = c.c_int
+    lib.si_set_tuning.argtypes = [i32, i32, i32]
     lib.si_status_string.restype = c.c_char_p
     lib.si_status_string.argtypes = [c.c_int]
     lib.si_version.restype = c.c_char_p
@@ -105,6 +107,12 @@ def select_sorts_rows(H: int, D: int, k: int) -> bool:
     """Whether the select kernel writes rows already sorted for these sizes
     (si_select_sorts_rows); otherwise indexer_topk adds the row-sort kernel."""
     return bool(load_library().si_select_sorts_rows(int(H), int(D), int(k)))
+
+
+def set_tuning(pool_entries: int = 0, cut_slack: int = 0, check_tiles: int = 0) -> None:
+    """Design parameters of the select kernel (si_set_tuning); 0 = default.
+    Results are the exact top-k for every setting; size workspaces after."""
+    _check(load_library().si_set_tuning(int(pool_entries), int(cut_slack), int(check_tiles)), "si_set_tuning")
 
 
 def set_sort_in_select(enable: bool) -> None:

@@ -36,6 +36,7 @@ struct SelectLaunch {
     bool smem_pool;      // candidate pools in shared memory (else gpool)
     int P;               // pool capacity per query
     int sort_e;          // unit-end row sort: 128 * sort_e keys per row, 0 = none
+    uint32_t check_tiles, cut_slack;
     uint64_t timeout_ns;
     uint64_t* gpool;
     unsigned long long* trace;
@@ -85,6 +86,8 @@ si_status launch_select_t(const SelectLaunch& a) {
     p.gpool = a.gpool;
     p.err = static_cast<uint32_t*>(a.ws);
     p.sort_e = a.sort_e;
+    p.check_tiles = a.check_tiles;
+    p.cut_slack = a.cut_slack;
     p.timeout_ns = a.timeout_ns;
     p.trace = a.trace;
 

@@ -108,6 +108,17 @@ constexpr int64_t kRowAlign = 256;
 // Whether the select kernel sorts each row at unit end (default) or leaves the
 // rows unordered for the separate row sort.
 std::atomic<bool> g_sort_in_select{true};
+// Design parameters set by si_set_tuning (0: the default).
+std::atomic<int> g_pool_entries{0}, g_cut_slack{0}, g_check_tiles{0};
+
+uint32_t check_tiles_in_use() {
+    const int c = g_check_tiles.load();
+    return c > 0 ? static_cast<uint32_t>(c) : si::kCheckTiles;
+}
+uint32_t cut_slack_in_use() {
+    const int c = g_cut_slack.load();
+    return c > 0 ? static_cast<uint32_t>(c) : si::kCompactSlack;
+}
 
 bool supported_h(int h) { return h == 8 || h == 16 || h == 32 || h == 64; }
 bool supported_d(int d) { return d == 64 || d == 128; }
@@ -137,16 +148,25 @@ struct PoolPlan {
 
 PoolPlan pool_plan(int H, int D, int k) {
     auto r32 = [](int x) { return (x + 31) / 32 * 32; };
-    const int spare = 2 * k < k + 768 ? 2 * k : k + 768;
-    const int min_p = r32(spare > k + 288 ? spare : k + 288);
     const uint32_t qt = 256u / static_cast<uint32_t>(H);
     const uint32_t fixed = select_smem(H, D, true, 0);  // everything but the pools
+    // room the appends need between two pool checks, plus survivors of a cut
+    const int need = k + static_cast<int>(4 * (32 * check_tiles_in_use() + 1)) + 28;
+    const int forced = g_pool_entries.load();
+    if (forced > 0) {  // si_set_tuning: a given capacity (at least `need`), in shared memory if it fits
+        const int p = r32(forced > need ? forced : need);
+        if (fixed + qt * static_cast<uint32_t>(p) * 8u <= kMaxDynSmem && p <= 65504) return {true, p};
+        return {false, p};
+    }
+    const int spare = 2 * k < k + 768 ? 2 * k : k + 768;
+    int min_p = r32(spare > k + 288 ? spare : k + 288);
+    if (min_p < need) min_p = r32(need);
     if (fixed + qt * static_cast<uint32_t>(min_p) * 8u <= kMaxDynSmem) {
         int p = static_cast<int>((kMaxDynSmem - fixed) / (qt * 8u)) / 32 * 32;
         if (p > 65504) p = 65504;  // pool counts are 16-bit fields
         return {true, p};
     }
-    return {false, r32(4 * k > k + 288 ? 4 * k : k + 288)};
+    return {false, r32(4 * k > min_p ? 4 * k : min_p)};
 }
 
 // Keys per thread of the unit-end row sort inside the select kernel (the
@@ -234,6 +254,8 @@ si_status launch_select(const void* q, const float* w, const void* kc, int64_t B
     a.smem_pool = pp.smem;
     a.P = pp.P;
     a.sort_e = (dense || !g_sort_in_select.load()) ? 0 : row_sort_e(H, D, k);
+    a.check_tiles = check_tiles_in_use();
+    a.cut_slack = cut_slack_in_use();
     a.timeout_ns = g_timeout_ns.load();
     a.gpool = pp.smem ? nullptr : reinterpret_cast<uint64_t*>(static_cast<uint8_t*>(ws) + kHeaderBytes);
 #ifdef SI_TRACE
@@ -403,6 +425,16 @@ int si_select_sorts_rows(int H_I, int d_I, int k) {
 }
 
 void si_set_sort_in_select(int enable) { g_sort_in_select.store(enable != 0); }
+
+si_status si_set_tuning(int pool_entries, int cut_slack, int check_tiles) {
+    if (pool_entries < 0 || pool_entries > 65504 || cut_slack < 0 || cut_slack > 4096 || check_tiles < 0 ||
+        check_tiles > 16)
+        return SI_ERR_INVALID_ARG;
+    g_pool_entries.store(pool_entries);
+    g_cut_slack.store(cut_slack);
+    g_check_tiles.store(check_tiles);
+    return SI_OK;
+}
 
 void si_set_timeout_ns(uint64_t ns) {
     if (ns > 0) g_timeout_ns.store(ns);

@@ -85,6 +85,8 @@ struct SelectParams {
     uint64_t* gpool;    // pools in global memory (per CTA QT*P), or nullptr
     uint32_t* err;      // device error word
     int sort_e;         // > 0: rows are written sorted, 128 * sort_e >= k keys per row; 0: unordered
+    uint32_t check_tiles;   // key tiles between two checks of the pools' fill (kCheckTiles by default)
+    uint32_t cut_slack;     // most entries above k an intermediate cut keeps (kCompactSlack by default)
     uint64_t timeout_ns;
     unsigned long long* trace;  // SI_TRACE builds only: [grid][kTraceWarps][kTraceSlots]
 };
@@ -147,12 +149,11 @@ struct SelCfg {
     static constexpr int NP = (4 / QH) < 1 ? 1 : ((4 / QH) > 2 ? 2 : 4 / QH);
 };
 
-// Extra entries an intermediate pool cut may keep above k (the cut at the end
-// of a unit is exact).
+// Defaults of two design parameters (SelectParams::cut_slack, check_tiles):
+// extra entries an intermediate pool cut may keep above k (the cut at the end
+// of a unit is exact), and key tiles between two checks of the pools' fill
+// (each check is a named barrier over the epilogue half).
 constexpr uint32_t kCompactSlack = 256;
-
-// Tiles between two checks of the pools' fill (each check is a named barrier
-// over the epilogue half).
 constexpr uint32_t kCheckTiles = 2;
 
 // Mbarrier slots.
@@ -1161,10 +1162,12 @@ __global__ void __launch_bounds__(SelCfg<H, D>::THREADS, 1)
         const int k = p.k;
         const uint32_t Pu = static_cast<uint32_t>(P);
         // An intermediate cut keeps at most k + cut_slack entries, which leaves
-        // every warp's sub-range more than kCheckTiles*32 free slots (P >= k + 288).
-        const uint32_t room = 4u * (32u * kCheckTiles + 1u);
+        // every warp's sub-range more than check_tiles*32 free slots (the host
+        // ensures P >= k + 4 * (32 * check_tiles + 1) + 28).
+        const uint32_t ct = p.check_tiles;
+        const uint32_t room = 4u * (32u * ct + 1u);
         const uint32_t cut_slack =
-            Pu > static_cast<uint32_t>(k) + room + kCompactSlack ? kCompactSlack : Pu - static_cast<uint32_t>(k) - room;
+            Pu > static_cast<uint32_t>(k) + room + p.cut_slack ? p.cut_slack : Pu - static_cast<uint32_t>(k) - room;
         uint32_t acc_it = 0, w_it = 0;
         bool bad = false;
         for (int64_t r = 0; r * G < U; ++r) {
@@ -1221,6 +1224,7 @@ __global__ void __launch_bounds__(SelCfg<H, D>::THREADS, 1)
             if (ui.ntiles > 0) load_w();
             SI_TR_ADD(kTrEpiUnit, tun0, tr_lead);
             bool need_acc = false, bad_acc = false;
+            uint32_t check_cd = ct;  // tiles until the next pool check
             for (int j = 0; j < ui.ntiles; ++j) {
                 const uint32_t buf = acc_it & 1u;
                 SI_TR_T0(tf0);
@@ -1263,19 +1267,20 @@ __global__ void __launch_bounds__(SelCfg<H, D>::THREADS, 1)
                             const uint32_t bal = __ballot_sync(0xffffffffu, pass);
                             if (pass) pool[(half * C::QH + q) * P + bw(q) + cw[q] + __popc(bal & lanemask_lt())] = key;
                             cw[q] += static_cast<uint32_t>(__popc(bal));
-                            need |= cw[q] + 32u * kCheckTiles > fw(q);
+                            need |= cw[q] + 32u * ct > fw(q);
                         }
                     }
                 }
                 SI_TR_ADD(kTrEpiAppend, tap0, tr_lead);
                 SI_TR_T0(tfl0);
-                // One barrier every kCheckTiles tiles (abort and cut requests are
-                // OR-reduced; sub-ranges keep room for kCheckTiles tiles of
+                // One barrier every check_tiles tiles (abort and cut requests are
+                // OR-reduced; sub-ranges keep room for check_tiles tiles of
                 // appends); two more only when some sub-range is nearly full or
                 // a wait failed.
                 need_acc |= need;
                 bad_acc |= !ok;
-                if ((j + 1) % kCheckTiles != 0 && j + 1 != ui.ntiles) continue;
+                if (--check_cd != 0 && j + 1 != ui.ntiles) continue;
+                check_cd = ct;
                 const bool bad_here = bad_acc || *abort_flag;
                 SI_TR_DEPI(static_cast<int>(need_acc));
                 SI_TR_ADD(kTrEpiFilter, tfl0, tr_lead);
@@ -1298,7 +1303,7 @@ __global__ void __launch_bounds__(SelCfg<H, D>::THREADS, 1)
                     for (int q = 0; q < C::QH; ++q) {
                         const uint32_t* c4 = cntw[half][q];
                         const uint32_t f = fw(q);
-                        constexpr uint32_t mg = 32u * kCheckTiles;
+                        const uint32_t mg = 32u * ct;
                         const bool cut = c4[0] + mg > f || c4[1] + mg > f || c4[2] + mg > f || c4[3] + mg > f;
                         if (!cut) continue;  // uniform over the half
                         uint64_t* pq = pool + (half * C::QH + q) * P;

@@ -139,3 +139,23 @@ def test_select_sorts_rows_host_arithmetic(lib):
             assert not si.select_sorts_rows(H, D, k), (H, D, k)
     assert not si.select_sorts_rows(64, 128, 0) and not si.select_sorts_rows(64, 128, 2049)
     assert not si.select_sorts_rows(48, 128, 64)
+
+
+def test_tuning_knob_host_side(lib):
+    """si_set_tuning: pool capacity, cut slack and check interval are
+    validated, change the workspace only through the pool capacity, and
+    reset to the defaults with zeros."""
+    base = si.workspace_bytes(1, 65536, 16384, 64, 128, 4, 512)
+    try:
+        si.set_tuning(pool_entries=1344)
+        assert si.workspace_bytes(1, 65536, 16384, 64, 128, 4, 512) == base  # fits shared memory
+        si.set_tuning(pool_entries=4096)
+        assert si.workspace_bytes(1, 65536, 16384, 64, 128, 4, 512) == 256 + 148 * 4 * 4096 * 8
+        si.set_tuning(check_tiles=6, cut_slack=64)
+        assert si.workspace_bytes(1, 65536, 16384, 64, 128, 4, 512) == base
+        for bad in [dict(pool_entries=-1), dict(check_tiles=17), dict(cut_slack=5000)]:
+            with pytest.raises(si.SIError):
+                si.set_tuning(**bad)
+    finally:
+        si.set_tuning()
+    assert si.workspace_bytes(1, 65536, 16384, 64, 128, 4, 512) == base
