@@ -382,6 +382,10 @@ def run_ours(args, world, rank, local):
         att = attention_measure(si, idx, wl, args, dev, stream, peaks, peak_src)
         att["indexer_plus_attention_ms"] = ms_per_step + att["ms"]
         line["csa_attention"] = att
+        prod = producers_measure(si, wl, args, dev, stream, peaks, peak_src)
+        line["csa_producers"] = prod
+        line["csa_step_ms"] = {"producers": prod["ms"], "indexer": ms_per_step, "attention": att["ms"],
+                               "total": prod["ms"] + ms_per_step + att["ms"]}
     # end to end through the public API with host buffers
     if not args.no_e2e:
         line["e2e"] = e2e_measure(si, q, w, kc, wl, args, world, dev, stream, flops_rank)
@@ -535,6 +539,37 @@ def attention_measure(si, idx, wl, args, dev, stream, peaks, peak_src):
             "indexer_plus_attention_ms": None}
 
 
+def producers_measure(si, wl, args, dev, stream, peaks, peak_src, d_model=4096):
+    """The indexer's inputs from hidden states (si_indexer_inputs): q, w and
+    the m:1 compressed keys by tcgen05 GEMMs, random weights, CUDA-event timed.
+    FLOPs: 2*B*S*d_model*(H_I*d_I + H_I) + 2*B*T*m*d_model*d_I."""
+    from streaming_top_indexer_b200 import synth
+    B, S, H, D, m = wl.B, wl.S, wl.H, wl.D, wl.m
+    x, w_q, w_w, w_k = synth.generate_hidden(B, S, d_model, H, D, m, seed=args.seed, device=dev)
+    q = torch.empty((B, S, H, D), dtype=torch.bfloat16, device=dev)
+    w = torch.empty((B, S, H), dtype=torch.float32, device=dev)
+    kc = torch.empty((B, S // m, D), dtype=torch.bfloat16, device=dev)
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    for _ in range(args.warmup):
+        si.indexer_inputs(x, w_q, w_w, w_k, H, D, m, q, w, kc, st, stream)
+    torch.cuda.synchronize(dev)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for e0, e1 in ev:
+        e0.record(stream)
+        si.indexer_inputs(x, w_q, w_w, w_k, H, D, m, q, w, kc, st, stream)
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    assert int(st.item()) == 0, "device error in the producers"
+    ms = statistics.mean(e0.elapsed_time(e1) for e0, e1 in ev)
+    flops = 2.0 * B * S * d_model * (H * D + H) + 2.0 * B * (S // m) * m * d_model * D
+    tflops = flops / (ms * 1e-3) / 1e12
+    del x, w_q, w_w, w_k, q, w, kc
+    return {"kernel": "gemm_kernel (q: BN=256, w: BN=64, kc: BN=128)", "d_model": d_model, "ms": ms,
+            "value": tflops, "unit": "TFLOP/s",
+            "roofline": {"bound": "tensor", "achieved": tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": tflops / peaks["bf16_tflops"], "peak_source": f"{peak_src} bf16 burst"}}
+
+
 def e2e_measure(si, q, w, kc, wl, args, world, dev, stream, flops_rank):
     """Same metric through indexer_topk_host: pinned host inputs copied in,
     outputs copied out, inside the timed region every step."""
@@ -574,7 +609,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--csa", action="store_true",
-                    help="also time CSA's sparse attention (128 heads, d=d_v=128) over the indexer's output")
+                    help="also time the rest of the CSA step: the producers of q, w, kc from hidden states "
+                         "(d_model 4096) and the sparse attention (128 heads, d=d_v=128) over the indexer's output")
     ap.add_argument("--sort-kernel", action="store_true",
                     help="sort rows in the separate row-sort kernel instead of inside the select kernel")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work")

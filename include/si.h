@@ -239,6 +239,28 @@ SI_API si_status si_sparse_attention(const void* q, const void* kcache, const vo
  * The workspace size depends on pool_entries: size it after the call. */
 SI_API si_status si_set_tuning(int pool_entries, int cut_slack, int check_tiles);
 
+/* The indexer's inputs from hidden states, with given weights (the paper has
+ * the indexer score queries against keys compressed at ratio m with a
+ * learned projection, StreamIndex: Memory-Bounded Compressed Sparse
+ * Attention via Streaming Top-k, Abstract, and gives neither the
+ * projections nor the compressor; this is the plainest reading):
+ *     q[b,t,h,:] = x[b,t,:] . W_q[h*d_I + (0..d_I), :]^T   bf16 [B,S,H_I,d_I]
+ *     w[b,t,h]   = x[b,t,:] . W_w[h, :]^T                   fp32 [B,S,H_I]
+ *     kc[b,s,:]  = (1/m) sum_{j<m} x[b,s*m+j,:] . W_k^T    bf16 [B,T,d_I], T = floor(S/m)
+ *   x:   bf16 [B,S,d_model];  W_q: bf16 [H_I*d_I, d_model];  W_w: bf16
+ *   [H_I, d_model];  W_k: bf16 [d_I, d_model] (the [out, in] layout).
+ *   Each output is one tcgen05 GEMM with fp32 accumulation; the key
+ *   compressor reads a group of m tokens as one row (the mean pooling is
+ *   part of the contraction).
+ *   status: a device word, set to 0 by the call and to SI_ERR_TIMEOUT if a
+ *   bounded device wait expired.
+ * Supported: d_model a multiple of 64; H_I a multiple of 4; d_I and H_I*d_I
+ * multiples of 8; B*S < 2^31.  All pointers 16-byte aligned (status 4).
+ * Allocates nothing; asynchronous on `stream`. */
+SI_API si_status si_indexer_inputs(const void* x, const void* w_q, const void* w_w, const void* w_k,
+                                   int64_t B, int64_t S, int d_model, int H_I, int d_I, int m,
+                                   void* q, float* w, void* kc, uint32_t* status, si_stream_t stream);
+
 /* Device-side wait limit, in nanoseconds, used by later calls (default 2 s). */
 SI_API void si_set_timeout_ns(uint64_t ns);
 

@@ -23,7 +23,7 @@ __all__ = [
     "SIError", "library_path", "load_library", "workspace_bytes", "indexer_topk",
     "select_topk", "sort_topk", "indexer_scores", "check_device_status",
     "selftest_timeout", "set_timeout_ns", "indexer_topk_host", "version", "select_sorts_rows",
-    "set_sort_in_select", "sparse_attention", "set_tuning",
+    "set_sort_in_select", "sparse_attention", "set_tuning", "indexer_inputs",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -71,6 +71,8 @@ def _declare(lib):
     lib.si_sparse_attention.restype = c.c_int
     lib.si_sparse_attention.argtypes = [vp, vp, vp, vp, i64, i64, i64, i32, i32, i32, i32, c.c_float, vp, vp, vp,
                                         vp]
+    lib.si_indexer_inputs.restype = c.c_int
+    lib.si_indexer_inputs.argtypes = [vp, vp, vp, vp, i64, i64, i32, i32, i32, i32, vp, vp, vp, vp, vp]
     lib.si_select_sorts_rows.restype = c.c_int
     lib.si_select_sorts_rows.argtypes = [i32, i32, i32]
     lib.si_set_sort_in_select.restype = None
@@ -368,3 +370,32 @@ def sparse_attention(q, kcache, vcache, idx, scale: float, out=None, lse=None, s
                                               DV, k, float(scale), out.data_ptr(), lse.data_ptr(),
                                               status.data_ptr(), _stream(stream)), "si_sparse_attention")
     return out, lse, status
+
+
+def indexer_inputs(x, w_q, w_w, w_k, H: int, D: int, m: int, q=None, w=None, kc=None, status=None, stream=None):
+    """q, w and kc of the indexer from hidden states (si_indexer_inputs).
+
+    x bf16 [B,S,d_model]; weights bf16 in [out, in] layout: w_q [H*D,
+    d_model], w_w [H, d_model], w_k [D, d_model].  Returns (q bf16 [B,S,H,D],
+    w fp32 [B,S,H], kc bf16 [B,S//m,D], status int32 [1] device word),
+    asynchronously on ``stream``.
+    """
+    _need(x, "x", torch.bfloat16, 3)
+    for name, t, rows in (("w_q", w_q, H * D), ("w_w", w_w, H), ("w_k", w_k, D)):
+        _need(t, name, torch.bfloat16, 2)
+        if tuple(t.shape) != (rows, x.shape[2]):
+            raise ValueError(f"{name} must be [{rows}, d_model]")
+    B, S, DM = x.shape
+    T = S // m
+    if q is None:
+        q = torch.empty((B, S, H, D), dtype=torch.bfloat16, device=x.device)
+    if w is None:
+        w = torch.empty((B, S, H), dtype=torch.float32, device=x.device)
+    if kc is None:
+        kc = torch.empty((B, T, D), dtype=torch.bfloat16, device=x.device)
+    if status is None:
+        status = torch.empty(1, dtype=torch.int32, device=x.device)
+    _check(load_library().si_indexer_inputs(x.data_ptr(), w_q.data_ptr(), w_w.data_ptr(), w_k.data_ptr(), B, S, DM,
+                                            H, D, m, q.data_ptr(), w.data_ptr(), kc.data_ptr(), status.data_ptr(),
+                                            _stream(stream)), "si_indexer_inputs")
+    return q, w, kc, status

@@ -173,3 +173,28 @@ def generate_attention(B: int, S: int, T: int, D: int = 128, DV: int = 128, seed
     kc = torch.randn((B, T, D), generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
     vc = torch.randn((B, T, DV), generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
     return q, kc, vc
+
+
+def generate_hidden(B: int, S: int, d_model: int, H: int, D: int, m: int, seed: int = 0, device="cpu"):
+    """Draw hidden states and random producer weights (no trained weights exist):
+    x bf16 [B,S,d_model] ~ N(0,1); W_q bf16 [H*D, d_model] ~ N(0, 1/(d_model*D)),
+    W_w bf16 [H, d_model] ~ N(0, 1/(d_model*H)), W_k bf16 [D, d_model]
+    ~ N(0, m/d_model), so that the projected q, w and kc have the spreads of
+    generate()'s inputs (N(0,1/D), N(0,1/H), N(0,1))."""
+    dev = torch.device(device)
+    g = torch.Generator(device=dev)
+    g.manual_seed(seed + 31337)
+    x = torch.empty((B, S, d_model), dtype=torch.bfloat16, device=dev)
+    rows = max(1, Q_BLOCK_ELEMS // d_model)
+    for b in range(B):
+        for s0 in range(0, S, rows):
+            s1 = min(S, s0 + rows)
+            x[b, s0:s1].copy_(torch.randn((s1 - s0, d_model), generator=g, device=dev, dtype=torch.float32))
+
+    def weight(rows_, std):
+        return (torch.randn((rows_, d_model), generator=g, device=dev, dtype=torch.float32) * std).to(torch.bfloat16)
+
+    w_q = weight(H * D, 1.0 / math.sqrt(d_model * D))
+    w_w = weight(H, 1.0 / math.sqrt(d_model * H))
+    w_k = weight(D, math.sqrt(m / d_model))
+    return x, w_q, w_w, w_k
