@@ -571,8 +571,9 @@ def producers_measure(si, wl, args, dev, stream, peaks, peak_src, d_model=4096):
 
 
 def e2e_measure(si, q, w, kc, wl, args, world, dev, stream, flops_rank):
-    """Same metric through indexer_topk_host: pinned host inputs copied in,
-    outputs copied out, inside the timed region every step."""
+    """Same metric through the C-ABI host-buffer call si_indexer_topk_host
+    (binding indexer_topk_host): pinned host inputs copied in, outputs copied
+    out, inside the timed region every step."""
     qh = q.cpu().pin_memory()
     wh = w.cpu().pin_memory()
     kch = kc.cpu().pin_memory()

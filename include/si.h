@@ -100,6 +100,39 @@ SI_API si_status si_indexer_topk_rows(const void* q, const float* w, const void*
                                int32_t* out_idx, float* out_score,
                                void* workspace, size_t workspace_bytes, si_stream_t stream);
 
+/* si_indexer_topk on HOST inputs and outputs, copies included (the call a
+ * user with host data makes).  Rows are computed in windows with
+ * si_indexer_topk_rows (rows select their keys independently: StreamIndex:
+ * Memory-Bounded Compressed Sparse Attention via Streaming Top-k, Abstract),
+ * last rows first.  While one window is computed on `stream`, the q and w rows
+ * of the next are copied in and the results of the previous one copied out,
+ * on two copy streams the library keeps per device.
+ *   q_h, w_h, kc_h: host q bf16 [B,S,H_I,d_I], w fp32 [B,S,H_I], kc bf16
+ *     [B,T,d_I]; idx_h, score_h: host outputs [B,S,k].  Page-locked host
+ *     memory lets the copies overlap the computation; pageable memory gives
+ *     the same results with serialised copies.
+ *   q_d, w_d, kc_d, idx_d, score_d: caller-owned device buffers of the same
+ *     shapes (the rules of si_indexer_topk apply to them); workspace as for
+ *     si_indexer_topk (its header is reset by this call).
+ *   chunks: number of row windows, 0 for the default min(32, max(1, S/2048));
+ *     windows hold a multiple of 256 rows (see si_host_window_rows).
+ *   The current device must be the one that owns `stream` and the buffers.
+ * Arguments are checked before anything is enqueued (the codes of
+ * si_indexer_topk, SI_ERR_INVALID_ARG for a null host pointer or chunks < 0).
+ * Everything is asynchronous: the host outputs are complete once `stream` is
+ * synchronised.  A later call, or other work on `stream`, may reuse the
+ * buffers: the copies in wait for the work queued on `stream` before. */
+SI_API si_status si_indexer_topk_host(const void* q_h, const float* w_h, const void* kc_h,
+                               int64_t B, int64_t S, int64_t T, int H_I, int d_I, int m, int k,
+                               int32_t* idx_h, float* score_h,
+                               void* q_d, float* w_d, void* kc_d, int32_t* idx_d, float* score_d,
+                               void* workspace, size_t workspace_bytes, int chunks, si_stream_t stream);
+
+/* Rows per window of si_indexer_topk_host for `chunks` windows: ceil(S /
+ * chunks) rounded down to a multiple of 256, at least 256 (0 for S <= 0);
+ * the last window ends at S. */
+SI_API int64_t si_host_window_rows(int64_t S, int chunks);
+
 /* First stage of si_indexer_topk alone: the fused scoring + selection kernel.
  * Does not reset the workspace header.  Where si_select_sorts_rows() is 1
  * for these sizes, the kernel also sorts each row at the end of its work

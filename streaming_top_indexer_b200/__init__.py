@@ -56,6 +56,10 @@ def _declare(lib):
         fn.argtypes = topk_args
     lib.si_indexer_topk_rows.restype = c.c_int
     lib.si_indexer_topk_rows.argtypes = topk_args[:10] + [i64, i64] + topk_args[10:]
+    lib.si_indexer_topk_host.restype = c.c_int
+    lib.si_indexer_topk_host.argtypes = topk_args[:12] + [vp, vp, vp, vp, vp, vp, sz, i32, vp]
+    lib.si_host_window_rows.restype = i64
+    lib.si_host_window_rows.argtypes = [i64, i32]
     lib.si_sort_topk.restype = c.c_int
     lib.si_sort_topk.argtypes = [vp, vp, i64, i32, vp]
     lib.si_indexer_scores.restype = c.c_int
@@ -268,34 +272,36 @@ def selftest_timeout(workspace, limit_ns: int, stream=None) -> int:
 
 
 def host_row_windows(S: int, chunks: int):
-    """Row windows of the pipelined host path: boundaries on multiples of 256
-    (the last window ends at S), about S/chunks rows each, no empty window."""
-    step = max(256, -(-S // max(1, chunks)) // 256 * 256)
+    """Row windows of si_indexer_topk_host, in row order: si_host_window_rows
+    rows each (a multiple of 256), the last window ending at S."""
+    step = int(load_library().si_host_window_rows(int(S), int(chunks)))
+    if step <= 0:
+        return []
     bounds = list(range(0, S, step)) + [S]
     return [(bounds[i], bounds[i + 1]) for i in range(len(bounds) - 1)]
 
 
 def indexer_topk_host(q, w, kc, m: int, k: int, device="cuda", buffers=None, stream=None, chunks=None):
-    """End-to-end call on host tensors: copies q, w, kc to the GPU, runs the
-    indexer and copies (idx, score) back into host tensors.
+    """End-to-end call on host tensors (si_indexer_topk_host): copies q, w, kc
+    to the GPU, runs the indexer and copies (idx, score) back into host
+    tensors, overlapped by row windows inside the library.
 
-    The rows are processed in windows (si_indexer_topk_rows), the last rows
-    (the most work, under the causal mask) first: while one window runs, the
-    inputs of the next are copied in and the results of the previous one
-    copied out, on two copy streams.  Host tensors should be pinned for the
-    copies to overlap.
-
-    ``chunks`` sets the number of windows (default: S/2048, at most 32).
+    Host tensors should be pinned for the copies to overlap.  ``chunks`` sets
+    the number of row windows (default: the library's, S/2048 capped at 32).
     ``buffers`` may hold preallocated device tensors ("q","w","kc","idx",
-    "score","ws"), pinned host outputs ("idx_h","score_h") and the copy
-    streams to reuse.  Returns (idx_h, score_h); everything is asynchronous
-    and complete once ``stream`` (default: torch's current stream) is
-    synchronised.
+    "score","ws") and pinned host outputs ("idx_h","score_h") to reuse; they
+    are created on first use.  Returns (idx_h, score_h), complete once
+    ``stream`` (default: torch's current stream) is synchronised.
     """
+    for t, n, dt, nd in ((q, "q", torch.bfloat16, 4), (w, "w", torch.float32, 3), (kc, "kc", torch.bfloat16, 3)):
+        if not isinstance(t, torch.Tensor) or t.is_cuda or t.dtype != dt or t.dim() != nd or not t.is_contiguous():
+            raise ValueError(f"{n} must be a contiguous {nd}-d {dt} host tensor")
     b = {} if buffers is None else buffers
     dev = torch.device(device)
     B, S, H, D = q.shape
     T = kc.shape[1]
+    if tuple(w.shape) != (B, S, H) or kc.shape[0] != B or kc.shape[2] != D:
+        raise ValueError(f"shape mismatch: q {tuple(q.shape)} w {tuple(w.shape)} kc {tuple(kc.shape)}")
     if "q" not in b:
         b["q"] = torch.empty(q.shape, dtype=torch.bfloat16, device=dev)
         b["w"] = torch.empty(w.shape, dtype=torch.float32, device=dev)
@@ -305,40 +311,15 @@ def indexer_topk_host(q, w, kc, m: int, k: int, device="cuda", buffers=None, str
         b["ws"] = torch.empty(workspace_bytes(B, S, T, H, D, m, k), dtype=torch.uint8, device=dev)
         b["idx_h"] = torch.empty((B, S, k), dtype=torch.int32, pin_memory=True)
         b["score_h"] = torch.empty((B, S, k), dtype=torch.float32, pin_memory=True)
-        b["s_in"] = torch.cuda.Stream(dev)
-        b["s_out"] = torch.cuda.Stream(dev)
     s = stream if stream is not None else torch.cuda.current_stream(dev)
-    s_in, s_out = b["s_in"], b["s_out"]
-    if chunks is None:  # measured at S=262,144: 8 -> 947, 16 -> 975, 32 -> 985 TFLOP/s end to end
-        chunks = max(1, min(32, S // 2048))
-    windows = host_row_windows(S, chunks)[::-1] if S > 0 else []
-    # The copy-in stream starts after everything already queued on `stream`
-    # (which includes the previous call's copy-out).
-    s_in.wait_stream(s)
-    with torch.cuda.stream(s_in):
-        b["kc"].copy_(kc, non_blocking=True)
-        in_done = []
-        for t0, t1 in windows:
-            b["q"][:, t0:t1].copy_(q[:, t0:t1], non_blocking=True)
-            b["w"][:, t0:t1].copy_(w[:, t0:t1], non_blocking=True)
-            ev = torch.cuda.Event()
-            ev.record(s_in)
-            in_done.append(ev)
-    out_ready = []
-    reset_device_status(b["ws"], s)
-    for (t0, t1), ev in zip(windows, in_done):
-        s.wait_event(ev)
-        indexer_topk_rows(b["q"], b["w"], b["kc"], m, k, t0, t1, b["idx"], b["score"], b["ws"], s)
-        done = torch.cuda.Event()
-        done.record(s)
-        out_ready.append(done)
-    with torch.cuda.stream(s_out):
-        for (t0, t1), ev in zip(windows, out_ready):
-            s_out.wait_event(ev)
-            b["idx_h"][:, t0:t1].copy_(b["idx"][:, t0:t1], non_blocking=True)
-            b["score_h"][:, t0:t1].copy_(b["score"][:, t0:t1], non_blocking=True)
-    s.wait_stream(s_out)
+    with torch.cuda.device(dev):
+        _check(load_library().si_indexer_topk_host(
+            q.data_ptr(), w.data_ptr(), kc.data_ptr() if T > 0 else None, B, S, T, H, D, m, k,
+            b["idx_h"].data_ptr(), b["score_h"].data_ptr(), b["q"].data_ptr(), b["w"].data_ptr(),
+            b["kc"].data_ptr() if T > 0 else None, b["idx"].data_ptr(), b["score"].data_ptr(), b["ws"].data_ptr(),
+            b["ws"].numel(), 0 if chunks is None else int(chunks), _stream(s)), "si_indexer_topk_host")
     return b["idx_h"], b["score_h"]
+
 
 def sparse_attention(q, kcache, vcache, idx, scale: float, out=None, lse=None, status=None, stream=None):
     """CSA sparse attention over the selected keys (si_sparse_attention).

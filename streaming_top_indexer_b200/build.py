@@ -26,7 +26,7 @@ ATTN_TRACE_LIB_PATH = os.path.join(LIB_DIR, "libsi_atrace.so")
 # The host library, one translation unit per H_I of the select kernel and the
 # sparse attention stage, compiled in parallel and linked into one library.
 SOURCES = [os.path.join(CSRC, f) for f in ("si_lib.cu", "si_select_h8.cu", "si_select_h16.cu", "si_select_h32.cu",
-                                           "si_select_h64.cu", "si_attn.cu", "si_proj.cu")]
+                                           "si_select_h64.cu", "si_attn.cu", "si_proj.cu", "si_host_io.cu")]
 BUILD_DIR = os.path.join(PKG, "_build")
 HEADERS = [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith(".cuh")] + [
     os.path.join(INCLUDE, "si.h")]

@@ -118,7 +118,7 @@ def test_row_window_arguments_before_any_cuda_call(lib):
     assert call_rows(lib, 0, 256, H=12) == 2
 
 
-def test_host_row_windows():
+def test_host_row_windows(lib):
     for S, chunks in [(262144, 8), (65536, 8), (2048, 8), (300, 8), (100, 4), (257, 1), (4096, 3)]:
         win = si.host_row_windows(S, chunks)
         assert win[0][0] == 0 and win[-1][1] == S
@@ -127,6 +127,31 @@ def test_host_row_windows():
         for a, b in win:
             assert a < b and a % 256 == 0 and (b % 256 == 0 or b == S)
         assert len(win) <= max(1, chunks) + 1
+        # rows per window: ceil(S / chunks) rounded down to a multiple of 256, at least 256
+        assert lib.si_host_window_rows(S, chunks) == max(256, -(-S // chunks) // 256 * 256)
+    assert lib.si_host_window_rows(0, 4) == 0 and si.host_row_windows(0, 4) == []
+    assert lib.si_host_window_rows(1000, 0) == 768  # chunks < 1 counts as one window
+
+
+def call_host(lib, **kw):
+    a = dict(qh=16, wh=16, kch=16, B=1, S=1000, T=250, H=64, D=128, m=4, k=4, ih=16, sh=16, q=16, w=16, kc=16,
+             oi=16, os_=16, ws=16, wsb=1 << 20, chunks=0)
+    a.update(kw)
+    return lib.si_indexer_topk_host(a["qh"], a["wh"], a["kch"], a["B"], a["S"], a["T"], a["H"], a["D"], a["m"],
+                                    a["k"], a["ih"], a["sh"], a["q"], a["w"], a["kc"], a["oi"], a["os_"], a["ws"],
+                                    a["wsb"], a["chunks"], None)
+
+
+def test_host_entry_arguments_before_any_cuda_call(lib):
+    """si_indexer_topk_host checks its host pointers, then every device-side
+    rule of si_indexer_topk, before anything is enqueued."""
+    for name in ("qh", "wh", "kch", "ih", "sh"):
+        assert call_host(lib, **{name: 0}) == 1, name
+    assert call_host(lib, kch=0, kc=0, T=0, chunks=-1) == 1    # negative window count
+    assert call_host(lib, q=0) == 1 and call_host(lib, oi=0) == 1
+    assert call_host(lib, H=12) == 2 and call_host(lib, k=2049) == 2
+    assert call_host(lib, w=20) == 3                              # misaligned device buffer
+    assert call_host(lib, wsb=8) == 4                             # workspace below si_workspace_bytes
 
 
 def test_select_sorts_rows_host_arithmetic(lib):

@@ -1,5 +1,6 @@
-"""Row windows (si_indexer_topk_rows) and the pipelined host path built on
-them: the same rows as the whole-problem call, bit for bit."""
+"""Row windows (si_indexer_topk_rows) and the pipelined host entry point
+built on them (si_indexer_topk_host): the same rows as the whole-problem
+call, bit for bit."""
 import pytest
 import torch
 
@@ -69,6 +70,53 @@ def test_pipelined_host_path_equals_device_call(chunks):
         assert si.check_device_status(bufs["ws"]) == 0
         assert torch.equal(idx_h, ref_idx.cpu())
         assert torch.equal(sc_h.view(torch.int32), ref_sc.cpu().view(torch.int32))
+
+
+@pytest.mark.parametrize("B,S,T,H,D,m,k", SHAPES)
+@pytest.mark.parametrize("pinned", [True, False])
+def test_host_entry_equals_device_call(B, S, T, H, D, m, k, pinned):
+    """Ragged S, several batches (strided row copies), k > T, T > S/m and
+    workspace pools, from page-locked and from pageable host memory."""
+    q, w, kc = inputs(B, S, T, H, D, m, k, seed=S + 11)
+    ref_idx, ref_sc = si.indexer_topk(q, w, kc, m, k)
+    qh, wh, kch = q.cpu(), w.cpu(), kc.cpu()
+    if pinned:
+        qh, wh, kch = qh.pin_memory(), wh.pin_memory(), kch.pin_memory()
+    bufs = {}
+    idx_h, sc_h = si.indexer_topk_host(qh, wh, kch, m, k, device=DEV, buffers=bufs, chunks=3)
+    torch.cuda.current_stream().synchronize()
+    assert si.check_device_status(bufs["ws"]) == 0
+    assert torch.equal(idx_h, ref_idx.cpu())
+    assert torch.equal(sc_h.view(torch.int32), ref_sc.cpu().view(torch.int32))
+
+
+def test_host_entry_with_no_keys_gives_padding():
+    B, S, H, D, m, k = 2, 600, 64, 128, 4, 8
+    q, w, _ = inputs(B, S, 4, H, D, m, k, seed=6)
+    kc = torch.empty((B, 0, D), dtype=torch.bfloat16)
+    idx_h, sc_h = si.indexer_topk_host(q.cpu().pin_memory(), w.cpu().pin_memory(), kc, m, k, device=DEV, chunks=2)
+    torch.cuda.current_stream().synchronize()
+    assert torch.all(idx_h == -1) and torch.all(torch.isneginf(sc_h))
+
+
+def test_host_entry_waits_for_work_queued_before():
+    """A second call may reuse the buffers at once: its copies in wait for the
+    first call's reads of them (both queued without a synchronisation)."""
+    B, S, T, H, D, m, k = 1, 2048, 512, 64, 128, 4, 64
+    q1, w1, kc1 = inputs(B, S, T, H, D, m, k, seed=21)
+    q2, w2, kc2 = inputs(B, S, T, H, D, m, k, seed=22)
+    r1 = si.indexer_topk(q1, w1, kc1, m, k)
+    r2 = si.indexer_topk(q2, w2, kc2, m, k)
+    h1 = [t.cpu().pin_memory() for t in (q1, w1, kc1)]
+    h2 = [t.cpu().pin_memory() for t in (q2, w2, kc2)]
+    bufs = {}
+    i1, s1 = si.indexer_topk_host(*h1, m, k, device=DEV, buffers=bufs, chunks=4)
+    torch.cuda.current_stream().synchronize()
+    assert torch.equal(i1, r1[0].cpu()) and torch.equal(s1, r1[1].cpu())
+    si.indexer_topk_host(*h1, m, k, device=DEV, buffers=bufs, chunks=4)
+    i2, s2 = si.indexer_topk_host(*h2, m, k, device=DEV, buffers=bufs, chunks=4)  # no synchronisation between
+    torch.cuda.current_stream().synchronize()
+    assert torch.equal(i2, r2[0].cpu()) and torch.equal(s2, r2[1].cpu())
 
 
 def test_windows_with_no_keys_give_padding():
