@@ -207,29 +207,15 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
 // Accumulates 32 TMEM columns (chunk c of the half) into the partial sums.
 // Column j of the half is head (j % H) of query (j / H); consecutive heads
 // are paired into one packed f32x2 FMA, pair p of a query goes to partial
-// sum p % NP.
-// How the ReLU of a head pair is computed.  max(x, 0) runs on the ALU pipe,
-// which has half the issue rate of the FMA pipe and also carries the
-// integer work; x + |x| = 2*relu(x) is one FADD on the FMA pipe (the abs is
-// an operand modifier).  Pairs computed the second way accumulate twice the
-// value into their own partial sums, which are halved at the end: scaling by
-// 2 is exact in binary floating point, so the scores are bit-identical either
-// way.  Mode 1 alternates the two ways by head pair (balancing the pipes),
-// mode 2 uses the FADD form for every pair.
-template <int NP>
-struct ReluPlan {
-    static constexpr int MODE = NP >= 2 ? 1 : 2;
-    // partial sum a holds doubled terms
-    static constexpr bool doubled(int a) { return MODE == 2 || (MODE == 1 && (a & 1)); }
-};
-
-__device__ __forceinline__ float relu_max(float x) { return fmaxf(x, 0.0f); }
-__device__ __forceinline__ float relu_twice(float x) { return x + fabsf(x); }
-
+// sum p % NP.  The ReLU of a head pair is one packed add, x + |x| =
+// 2*max(x, 0) (exact in binary floating point), so the partial sums hold
+// twice the weighted sums and are halved at the end, also exact unless a
+// partial sum is subnormal or beyond half the fp32 range: the scores equal
+// sum_h w_h * max(x_h, 0) summed in the same order.  Measured against a mix
+// of max() on the ALU pipe and scalar adds: equal or up to 2 % faster.
 template <int H, int QH, int NP, int CG>
 __device__ __forceinline__ void accumulate_chunk(const uint32_t (&r)[32], int c, const float (&wr)[CG],
                                                  float2 (&acc)[QH][NP]) {
-    using RP = ReluPlan<NP>;
 #pragma unroll
     for (int i = 0; i < 32; i += 4) {
         const int col = c * 32 + i;
@@ -239,10 +225,8 @@ __device__ __forceinline__ void accumulate_chunk(const uint32_t (&r)[32], int c,
         const int p0 = (h / 2) % NP, p1 = (h / 2 + 1) % NP;
         const float a0 = __uint_as_float(r[i]), a1 = __uint_as_float(r[i + 1]);
         const float a2 = __uint_as_float(r[i + 2]), a3 = __uint_as_float(r[i + 3]);
-        const float2 x01 = RP::doubled(p0) ? make_float2(relu_twice(a0), relu_twice(a1))
-                                           : make_float2(relu_max(a0), relu_max(a1));
-        const float2 x23 = RP::doubled(p1) ? make_float2(relu_twice(a2), relu_twice(a3))
-                                           : make_float2(relu_max(a2), relu_max(a3));
+        const float2 x01 = __fadd2_rn(make_float2(a0, a1), make_float2(fabsf(a0), fabsf(a1)));
+        const float2 x23 = __fadd2_rn(make_float2(a2, a3), make_float2(fabsf(a2), fabsf(a3)));
         acc[q][p0] = __ffma2_rn(make_float2(w4.x, w4.y), x01, acc[q][p0]);
         acc[q][p1] = __ffma2_rn(make_float2(w4.z, w4.w), x23, acc[q][p1]);
     }
@@ -276,10 +260,7 @@ __device__ __forceinline__ void half_scores(uint32_t taddr, const float (&wr)[32
     for (int q = 0; q < QH; ++q) {
         float part[NP];
 #pragma unroll
-        for (int a = 0; a < NP; ++a) {
-            part[a] = acc[q][a].x + acc[q][a].y;
-            if (ReluPlan<NP>::doubled(a)) part[a] *= 0.5f;
-        }
+        for (int a = 0; a < NP; ++a) part[a] = (acc[q][a].x + acc[q][a].y) * 0.5f;  // undo x + |x| = 2 relu(x)
 #pragma unroll
         for (int w = 1; w < NP; w *= 2)
 #pragma unroll
