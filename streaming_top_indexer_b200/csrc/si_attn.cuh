@@ -11,17 +11,24 @@
 //
 // One CTA per SM, a persistent loop over query rows; every row costs the same
 // (ceil(k/64) key chunks).  Per row the 128 heads are the MMA's M (one TMEM
-// lane each); per chunk of 64 selected keys:
-//   S   = Q K^T      tcgen05.mma M=128 N=64  K=d    (fp32 in TMEM)
+// lane each); per pair of chunks of 64 selected keys (per chunk when the
+// count is odd):
+//   S   = Q K^T      tcgen05.mma M=128 N=128 K=d    (fp32 in TMEM; N=64 alone)
+// and per chunk:
 //   P   = softmax    one thread per head, online, bf16 into shared memory
 //   O  += P V        tcgen05.mma M=128 N=dv K=64    (V as an MN-major operand)
+// Each tcgen05.mma instruction costs the issuing thread about 100 cycles
+// whatever its N, so S over two chunks at once halves the S issue time
+// (16 instructions per 128 keys in all, against 24 one chunk at a time).
 // Roles (384 threads):
 //   warp 0      TMA: q tiles (one buffer per softmax group);
 //   warp 1      TMEM allocation and the MMA issuer (an event loop: S and,
 //               per softmax group, P V are each issued as soon as their
 //               inputs are ready);
 //   warps 2-3   the chunks' K and V rows, gathered by index with 16-byte
-//               cp.async copies into an NST-stage ring, half of each chunk's
+//               cp.async copies into an NST-stage ring (NST even; K is laid
+//               out sub-tile-major so that stages 2j and 2j+1 form one
+//               128-row operand), half of each chunk's
 //               rows per warp (the selected rows are scattered 128- or 256-byte rows:
 //               measured, TMA gather4 moved them at about 10 GB/s per SM, one
 //               128-byte row segment every ~12 ns, which bounded the kernel);
@@ -92,17 +99,22 @@ struct AttnCfg {
     // everything but the K/V ring: two q buffers, one P buffer per group, alignment slack
     static constexpr uint32_t FIXED = 2 * Q_BYTES + 2 * P_BYTES + 1024 + STATIC_MAX;
     static constexpr int NST_FIT = static_cast<int>((SMEM_LIMIT - FIXED) / (K_BYTES + V_BYTES));
-    static constexpr int NST = NST_FIT > 6 ? 6 : NST_FIT;   // K/V ring stages
+    // K/V ring stages, even: a chunk pair takes stages 2j, 2j+1
+    static constexpr int NST = (NST_FIT > 6 ? 6 : NST_FIT) & ~1;
     static_assert(NST >= 2, "shared memory budget");
     static constexpr uint32_t OFF_Q = 0;                // [2] by softmax group
     static constexpr uint32_t OFF_P = OFF_Q + 2 * Q_BYTES;   // [group]
+    // K ring: [d/64 sub-tiles][NST stages][64 keys x 128 bytes], so that two
+    // adjacent stages of one sub-tile are 128 consecutive rows
     static constexpr uint32_t OFF_K = OFF_P + 2 * P_BYTES;
+    static constexpr uint32_t K_SUB_STRIDE = NST * KV_SUB;
     static constexpr uint32_t OFF_V = OFF_K + NST * K_BYTES;
     static constexpr uint32_t DYN_BYTES = OFF_V + NST * V_BYTES + 1024;
     static constexpr int THREADS = 384;
-    // Registers: every role fits the launch allocation (168 per thread)
-    // without spills (ptxas -v); a setmaxnreg re-split between the control
-    // and softmax warpgroups made ptxas spill around it, so there is none.
+    // Registers: every role runs in the launch allocation (168 per thread;
+    // ptxas -v reports about 56 bytes of spill stores); a setmaxnreg re-split
+    // between the control and softmax warpgroups made ptxas spill much more
+    // around it, so there is none.
     static constexpr uint32_t TMEM_COLS = 512;
     // TMEM: group w: S[w][2] at columns 128w + {0, 64}; O[w] at 256 + w*DV
     static constexpr uint32_t TM_O = 256;
@@ -139,10 +151,13 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return r;
 }
 
-// The CTA's work items in issue order: its rows i = 0 .. nrows-1 (query row
-// blockIdx.x + i * gridDim.x) go in pairs (2p, 2p+1), one per softmax group,
-// and the two rows' chunks alternate: (2p, 0), (2p+1, 0), (2p, 1), ...  An odd
-// last row runs alone.
+// The CTA's work items (one 64-key chunk each) in issue order: its rows
+// i = 0 .. nrows-1 (query row blockIdx.x + i * gridDim.x) go in pairs
+// (2p, 2p+1), one per softmax group, and the two rows' chunks alternate by
+// chunk pairs: (2p, 0), (2p, 1), (2p+1, 0), (2p+1, 1), (2p, 2), (2p, 3), ...;
+// with an odd chunk count the last chunks follow alone, (2p, NC-1),
+// (2p+1, NC-1).  An odd last row runs alone, its chunks in order.  Every
+// chunk pair starts at an even item, so its two ring stages are adjacent.
 struct AttnItem {
     int64_t i;   // row ordinal in the CTA
     int c;       // chunk of the row
@@ -155,9 +170,16 @@ __device__ __forceinline__ AttnItem attn_item(int64_t g, int64_t nrows, int NC) 
     const int64_t pair_items = 2 * static_cast<int64_t>(NC);
     const int64_t base = (nrows >> 1) * pair_items;
     if (g < base) {
-        const int64_t p = g / pair_items, r = g % pair_items;
-        it.c = static_cast<int>(r >> 1);
-        it.w = static_cast<int>(r & 1);
+        const int64_t p = g / pair_items;
+        const int r = static_cast<int>(g % pair_items);
+        const int full = (NC >> 1) * 4;  // items of the two rows' complete chunk pairs
+        if (r < full) {
+            it.w = (r >> 1) & 1;
+            it.c = (r >> 2) * 2 + (r & 1);
+        } else {
+            it.w = r - full;
+            it.c = NC - 1;
+        }
         it.i = 2 * p + it.w;
     } else {
         it.i = nrows - 1;
@@ -166,6 +188,16 @@ __device__ __forceinline__ AttnItem attn_item(int64_t g, int64_t nrows, int NC) 
     }
     it.lc = (it.i >> 1) * NC + it.c;
     return it;
+}
+
+// Item index of chunk c of row ordinal i (the inverse of attn_item).
+__device__ __forceinline__ int64_t attn_item_of(int64_t i, int c, int64_t nrows, int NC) {
+    const int64_t pair = i >> 1;
+    if (pair == (nrows >> 1)) return (nrows >> 1) * 2 * NC + c;  // the odd last row, alone
+    const int w = static_cast<int>(i & 1);
+    const int64_t base = pair * 2 * NC;
+    if (c < (NC & ~1)) return base + (c >> 1) * 4 + w * 2 + (c & 1);
+    return base + (NC >> 1) * 4 + w;
 }
 
 template <int D, int DV>
@@ -268,8 +300,10 @@ __global__ void __launch_bounds__(AttnCfg<D, DV>::THREADS, 1)
                 const int j = it.c * C::NK + half * 32 + lane;
                 return j < p.k ? p.idx[(blockIdx.x + it.i * G) * p.k + j] : -1;
             };
-            // copies of one operand (DD = d for K, d_v for V) of the warp's 32 rows
-            auto copy_rows = [&](const uint16_t* cache, uint32_t dst_stage, int key, int64_t kbase, int dd) {
+            // copies of one operand (DD = d for K, d_v for V) of the warp's 32 rows;
+            // 64-column sub-tile cc of the stage starts at dst_stage + cc * sub_stride
+            auto copy_rows = [&](const uint16_t* cache, uint32_t dst_stage, uint32_t sub_stride, int key, int64_t kbase,
+                                 int dd) {
                 const int ppr = dd / 8;              // 16-byte pieces per row
                 const int rpi = 32 / ppr;            // rows per warp instruction
                 const int pc = lane % ppr, cc = pc >> 3, c16 = pc & 7;
@@ -277,7 +311,7 @@ __global__ void __launch_bounds__(AttnCfg<D, DV>::THREADS, 1)
                     const int lr = it2 * rpi + lane / ppr;          // row within the warp's 32
                     const int r = half * 32 + lr;                   // row within the chunk
                     const int kr = __shfl_sync(0xffffffffu, key, lr);
-                    const uint32_t dst = dst_stage + cc * C::KV_SUB + static_cast<uint32_t>(r >> 3) * 1024u +
+                    const uint32_t dst = dst_stage + cc * sub_stride + static_cast<uint32_t>(r >> 3) * 1024u +
                                          static_cast<uint32_t>(r & 7) * 128u +
                                          (static_cast<uint32_t>(c16 ^ (r & 7)) << 4);
                     cp_async_16(dst, cache + (kbase + kr) * dd + pc * 8);
@@ -292,8 +326,8 @@ __global__ void __launch_bounds__(AttnCfg<D, DV>::THREADS, 1)
                 const int key = valid ? ent : 0;  // padding reads key 0, masked in the softmax
                 const uint32_t m = __ballot_sync(0xffffffffu, valid);
                 if (lane == 0) masks[st][half] = m;  // published by the release of this warp's arrive
-                copy_rows(p.kcache, sbase + C::OFF_K + st * C::K_BYTES, key, kbase, D);
-                copy_rows(p.vcache, sbase + C::OFF_V + st * C::V_BYTES, key, kbase, DV);
+                copy_rows(p.kcache, sbase + C::OFF_K + st * C::KV_SUB, C::K_SUB_STRIDE, key, kbase, D);
+                copy_rows(p.vcache, sbase + C::OFF_V + st * C::V_BYTES, C::KV_SUB, key, kbase, DV);
                 cp_async_commit();
                 if (half == 0 && lane == 0) SI_AT(0, g, 3);
             };
@@ -350,12 +384,14 @@ __global__ void __launch_bounds__(AttnCfg<D, DV>::THREADS, 1)
             __syncwarp();
         } else if (warp == 1) {
             // -------------------------------------------- MMA issuer
-            // An event loop: S of the next chunk (in issue order) and, for
-            // each softmax group, P V of its next chunk are issued as soon as
-            // their inputs are ready (tested without blocking).  The groups'
-            // O accumulations are independent, so neither waits for the other.
+            // An event loop: S of the next chunk pair (or lone chunk, in issue
+            // order) and, for each softmax group, P V of its next chunk are
+            // issued as soon as their inputs are ready (tested without
+            // blocking).  The groups' O accumulations are independent, so
+            // neither waits for the other.
             if (lane == 0) {
                 constexpr uint32_t idesc_s = idesc_bf16_f32(C::HA, C::NK);
+                constexpr uint32_t idesc_s2 = idesc_bf16_f32(C::HA, 2 * C::NK);
                 constexpr uint32_t idesc_o = idesc_bf16_f32_bmn(C::HA, DV);
                 // descriptors of the operand tiles' first K step; a K step of 16
                 // adds 32 bytes (K-major) or 2048 bytes (MN-major V) to the start
@@ -377,29 +413,39 @@ __global__ void __launch_bounds__(AttnCfg<D, DV>::THREADS, 1)
                     bool progress = false;
                     if (gs < total) {
                         const uint32_t st = static_cast<uint32_t>(gs % C::NST), u = static_cast<uint32_t>(gs / C::NST);
+                        // chunks c and c+1 of the row at items gs, gs+1 (stages st, st+1).
+                        // Pairs need an even chunk count: then a pair's first chunk has an
+                        // even group ordinal lc and takes the first of the group's two S
+                        // halves, so the pair's 128 columns are the group's S region.
+                        const bool two = (NC & 1) == 0 && (is.c & 1) == 0;
                         const int sb = is.w * 2 + static_cast<int>(is.lc & 1);
-                        const int64_t su = is.lc >> 1;
+                        const int64_t su = is.lc >> 1;  // uses of the S half (both halves for a pair)
                         const bool ready =
                             (is.c != 0 || mbar_test_wait(bar(kAQFull + is.w), static_cast<uint32_t>(is.i >> 1) & 1u)) &&
                             mbar_test_wait(bar(kAKFull + st), u & 1u) &&
-                            (su == 0 || mbar_test_wait(bar(kASFree + sb), static_cast<uint32_t>(su - 1) & 1u));
+                            (!two || mbar_test_wait(bar(kAKFull + st + 1), u & 1u)) &&
+                            (su == 0 || (mbar_test_wait(bar(kASFree + sb), static_cast<uint32_t>(su - 1) & 1u) &&
+                                         (!two || mbar_test_wait(bar(kASFree + sb + 1),
+                                                                 static_cast<uint32_t>(su - 1) & 1u))));
                         if (ready) {
                             SI_AT(1, gs, 0);
                             tc_fence_after();
                             const uint32_t d_tmem = tmem_base + is.w * 128 + static_cast<uint32_t>(is.lc & 1) * C::NK;
                             const uint64_t da = dq0 + ((is.w * C::Q_BYTES) >> 4);
-                            const uint64_t db = dk0 + ((st * C::K_BYTES) >> 4);
+                            const uint64_t db = dk0 + ((st * C::KV_SUB) >> 4);
 #pragma unroll
                             for (int kk = 0; kk < D / 16; ++kk) {
                                 const uint32_t off = ((kk / 4) * C::Q_SUB + (kk % 4) * 32) >> 4;
-                                const uint32_t offk = ((kk / 4) * C::KV_SUB + (kk % 4) * 32) >> 4;
-                                umma_bf16(d_tmem, da + off, db + offk, idesc_s, kk > 0 ? 1u : 0u);
+                                const uint32_t offk = ((kk / 4) * C::K_SUB_STRIDE + (kk % 4) * 32) >> 4;
+                                umma_bf16(d_tmem, da + off, db + offk, two ? idesc_s2 : idesc_s, kk > 0 ? 1u : 0u);
                             }
                             umma_commit(bar(kASFull + sb));
-                            if (is.c == NC - 1) umma_commit(bar(kAQEmpty + is.w));
+                            if (two) umma_commit(bar(kASFull + sb + 1));
+                            if (is.c + (two ? 1 : 0) == NC - 1) umma_commit(bar(kAQEmpty + is.w));
                             SI_AT(1, gs, 1);
                             issued = progress = true;
-                            if (++gs < total) is = attn_item(gs, nrows, NC);
+                            gs += two ? 2 : 1;
+                            if (gs < total) is = attn_item(gs, nrows, NC);
                         }
                     }
 #pragma unroll
@@ -408,8 +454,7 @@ __global__ void __launch_bounds__(AttnCfg<D, DV>::THREADS, 1)
                         const int64_t i = pr[w];
                         const int c = pc[w];
                         // the chunk's place in issue order, and the group's own ordinal
-                        const int64_t pair = i >> 1;
-                        const int64_t g = pair == (nrows >> 1) ? (nrows >> 1) * 2 * NC + c : pair * 2 * NC + 2 * c + w;
+                        const int64_t g = attn_item_of(i, c, nrows, NC);
                         if (g >= gs) continue;  // its S is not issued yet
                         const int64_t lc = (i >> 1) * NC + c, ouse = i >> 1;
                         const bool ready = mbar_test_wait(bar(kAPFull + w), static_cast<uint32_t>(lc) & 1u) &&
@@ -470,10 +515,8 @@ __global__ void __launch_bounds__(AttnCfg<D, DV>::THREADS, 1)
             const int64_t row = blockIdx.x + i * G;
             float m_run = NEG_INF, l_run = 0.0f;
             for (int c = 0; c < NC; ++c) {
-                // global item index of (i, c): pairs before, then the interleave
-                const int64_t pair = i >> 1;
-                const bool alone = (pair == (nrows >> 1));
-                const int64_t g = alone ? (nrows >> 1) * 2 * NC + c : pair * 2 * NC + 2 * c + w;
+                // global item index of (i, c)
+                const int64_t g = attn_item_of(i, c, nrows, NC);
                 const int64_t lc = (i >> 1) * NC + c;
                 const int sb = w * 2 + static_cast<int>(lc & 1);
                 const uint32_t su = static_cast<uint32_t>(lc >> 1);
