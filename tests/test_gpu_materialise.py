@@ -74,6 +74,49 @@ def test_streaming_equals_materialise_with_ties():
     assert torch.equal(got_sc.view(torch.int32), ref_sc.view(torch.int32))
 
 
+def materialise_topk_chunked(dense, m, k, rows=4096):
+    """materialise_topk's selection on given dense scores, sorted in blocks of
+    rows (the full-size cases hold a [S, T] fp32 tensor of gigabytes)."""
+    B, S, T = dense.shape
+    idx = torch.full((B, S, k), -1, dtype=torch.int32, device=dense.device)
+    score = torch.full((B, S, k), float("-inf"), dtype=torch.float32, device=dense.device)
+    kk = min(k, T)
+    for b in range(B):
+        for t0 in range(0, S, rows):
+            t1 = min(S, t0 + rows)
+            blk = dense[b, t0:t1]
+            sc = torch.where(torch.isnan(blk), torch.full_like(blk, float("-inf")), blk)
+            order = torch.sort(-sc, dim=-1, stable=True).indices[:, :kk]
+            idx[b, t0:t1, :kk] = order.to(torch.int32)
+            score[b, t0:t1, :kk] = torch.gather(sc, -1, order)
+            del sc, order
+    t = torch.arange(S, device=dense.device)
+    vis = torch.clamp((t + 1) // m, max=T)
+    pad = torch.arange(k, device=dense.device)[None, :] >= vis[:, None]
+    idx[:, pad] = -1
+    score[:, pad] = float("-inf")
+    return idx, score
+
+
+@pytest.mark.parametrize("B,S,T,H,D,m,k,kind", [
+    (1, 65536, 16384, 64, 128, 4, 512, "normal"),     # the V4-Flash-like shape, every row
+    (1, 32768, 8192, 64, 128, 4, 2048, "tieheavy"),   # workspace pools, many equal scores
+])
+def test_streaming_equals_materialise_at_full_size(B, S, T, H, D, m, k, kind):
+    """Every row of a full-size problem, bit for bit: the streaming result
+    against a stable sort of the dense scores (thousands of pool cuts and
+    unit-end selects per launch)."""
+    wl = synth.Workload("mat_full", B, S, m, H, D, k, kind)
+    q, w, kc = synth.generate(wl, seed=11, device=DEV, T=T)
+    got_idx, got_sc = gh.gpu_topk(q, w, kc, m, k)
+    dense = si.indexer_scores(q, w, kc, m)
+    del q, w, kc
+    ref_idx, ref_sc = materialise_topk_chunked(dense, m, k)
+    del dense
+    assert torch.equal(got_idx, ref_idx)
+    assert torch.equal(got_sc.view(torch.int32), ref_sc.view(torch.int32))
+
+
 def per_head_materialise_topk(q, w, kc, m, k):
     """The pages' baseline in its own form (StreamIndex, Abstract: public CSA
     code materialises the [B,S,H_I,T] fp32 score tensor before the top-k):
