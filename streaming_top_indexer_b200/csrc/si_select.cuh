@@ -550,11 +550,14 @@ __device__ __forceinline__ int half_samples(const uint64_t* pool, const PoolRegi
 //     keys is gathered into `big` (up to big_cap keys, shared memory) and
 //     the same select picks the k-th key among them.  Any larger bracket
 //     falls back to the radix select.
+//  When a sample qualifies directly, `counts_out` (if given) gets the
+//  per-warp counts of keys at or above it, which that counting pass left in
+//  shared memory (they stay valid until the half's next exchange).
 template <bool BIG = false, typename Keys>
 __device__ __forceinline__ uint64_t half_select_bound(const Keys& keys, const uint64_t* pool, const PoolRegions& rg,
                                                       int k, uint32_t max_keep, CutScratch& cs, int tid,
                                                       uint32_t bar_id, uint32_t& phase, uint64_t* big = nullptr,
-                                                      int big_cap = 0) {
+                                                      int big_cap = 0, const uint32_t** counts_out = nullptr) {
     const int n = rg.total();
     const int ns = half_samples(pool, rg, cs, tid, bar_id);
     // c(r) = #(keys >= srt[r]) grows with r; c(-1) = 0 (no bound), c(ns) = n (bound 0)
@@ -566,7 +569,10 @@ __device__ __forceinline__ uint64_t half_select_bound(const Keys& keys, const ui
     uint32_t c_lo = 0, c_hi = static_cast<uint32_t>(n);
     for (int it = 0; it < 8; ++it) {
         const uint32_t c = half_count_ge(keys, cs.srt[r], cs, tid, bar_id, phase);
-        if (c >= ku && c <= max_keep) return cs.srt[r];
+        if (c >= ku && c <= max_keep) {
+            if (counts_out) *counts_out = cs.rcnt[(phase - 1u) & 1u];  // the buffer half_sum just used
+            return cs.srt[r];
+        }
         if (c < ku) {
             lo_r = r;
             c_lo = c;
@@ -785,10 +791,13 @@ __device__ __forceinline__ uint32_t half_walk_kept(const uint64_t* pool, const P
 }
 
 // half_walk_kept for keys held in registers: one barrier, then each thread
-// emits its kept keys (safe in place: every key was read before).
+// emits its kept keys (safe in place: every key was read before).  With
+// `known` (the per-warp counts of keys >= L, from the counting pass that
+// chose L), the exchange and its barrier are skipped.
 template <typename Emit>
 __device__ __forceinline__ uint32_t half_walk_reg(const RegKeys& rk, uint64_t L, CutScratch& cs, int tid,
-                                                  uint32_t bar_id, uint32_t& phase, Emit emit) {
+                                                  uint32_t bar_id, uint32_t& phase, Emit emit,
+                                                  const uint32_t* known = nullptr) {
     const int lane = tid & 31, wq = tid >> 5;
     uint32_t keep = 0, mine = 0;
 #pragma unroll
@@ -799,10 +808,14 @@ __device__ __forceinline__ uint32_t half_walk_reg(const RegKeys& rk, uint64_t L,
     }
     uint32_t wtot;
     const uint32_t excl = warp_prefix_small(mine, lane, wtot);  // mine <= kRegKeys < 32
-    uint32_t* rc = cs.rcnt[phase & 1u];
-    ++phase;
-    if (lane == 0) rc[wq] = wtot;
-    bar_sync(bar_id, 128);
+    const uint32_t* rc = known;
+    if (!known) {
+        uint32_t* mine_rc = cs.rcnt[phase & 1u];
+        ++phase;
+        if (lane == 0) mine_rc[wq] = wtot;
+        bar_sync(bar_id, 128);
+        rc = mine_rc;
+    }
     uint32_t pos = excl, total = 0;
 #pragma unroll
     for (int w = 0; w < 4; ++w) {
@@ -831,10 +844,13 @@ static __device__ __noinline__ uint64_t cut_pool(uint64_t* pq, PoolRegions rg, i
     if (rg.total() <= 128 * kRegKeys) {
         RegKeys rk;
         rk.load(pq, rg, tid);
+        // when a sample qualifies, its counting pass already has the per-warp
+        // counts the pack needs (and every key is in registers: safe in place)
+        const uint32_t* known = nullptr;
         if (rk.n > k)
-            L = big ? half_select_bound<true>(rk, pq, rg, k, max_keep, cs, tid, bar_id, phase, big, big_cap)
-                    : half_select_bound(rk, pq, rg, k, max_keep, cs, tid, bar_id, phase);
-        kept = half_walk_reg(rk, L, cs, tid, bar_id, phase, pack);
+            L = big ? half_select_bound<true>(rk, pq, rg, k, max_keep, cs, tid, bar_id, phase, big, big_cap, &known)
+                    : half_select_bound(rk, pq, rg, k, max_keep, cs, tid, bar_id, phase, nullptr, 0, &known);
+        kept = half_walk_reg(rk, L, cs, tid, bar_id, phase, pack, known);
     } else {
         const StreamKeys sk{pq, rg};
         uint32_t m = 0;
