@@ -104,8 +104,26 @@ def build(force: bool = False, verbose: bool = False, extra=(), trace: bool = Fa
     return out
 
 
+CUT_BENCH_SRC = os.path.join(CSRC, "si_cut_bench.cu")
+CUT_BENCH_PATH = os.path.join(BUILD_DIR, "si_cut_bench")  # microbenchmark of the pool cut (development tool)
+
+
+def build_cut_bench(verbose: bool = False) -> str:
+    """The pool-cut microbenchmark executable (not part of the library)."""
+    os.makedirs(BUILD_DIR, exist_ok=True)
+    cmd = [nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, CUT_BENCH_SRC, "-o", CUT_BENCH_PATH]
+    if verbose:
+        print(" ".join(cmd), file=sys.stderr)
+    res = subprocess.run(cmd, capture_output=True, text=True)
+    if res.returncode != 0:
+        raise RuntimeError(f"nvcc failed on si_cut_bench.cu ({res.returncode}):\n{res.stderr[-8000:]}")
+    return CUT_BENCH_PATH
+
+
 if __name__ == "__main__":
-    if "--attn-trace" in sys.argv:
+    if "--cut-bench" in sys.argv:
+        print(build_cut_bench(verbose=True))
+    elif "--attn-trace" in sys.argv:
         print(build(verbose=True, extra=["-DSI_ATTN_TRACE"], out=ATTN_TRACE_LIB_PATH))
     elif "--fault-test" in sys.argv:
         print(build_fault_test(force=True, verbose=True))
